@@ -1,0 +1,411 @@
+"""Benchmark of the MoE-layer forward pass on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one moe_forward (router, top-k, permute, gather, gate/up GEMM,
+down GEMM, combine) over one batch of the workload, inputs resident in HBM.
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch
+(seeded by rank) against the same weights: data-parallel replicas, no
+collective on the data path ("scaling": "weak").  --impl reference times the
+CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; % of HBM (decode) / tensor-core (prefill) roofline"
+DEFAULT_WORKLOAD = "step3_decode"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------- algorithmic work
+
+def algorithmic(w, valid_tokens: int, offsets, k: int):
+    """Bytes and flops the method must move / compute (touched experts only),
+    per step and for the gate/up GEMM alone."""
+    import numpy as np
+    counts = np.diff(np.asarray(offsets))
+    U = int((counts > 0).sum())
+    routed_rows = int(counts.sum())
+    H, I, E, S, Is = w.H, w.I, w.E, w.S, (w.Is if w.S else 0)
+    wb = 2 if w.wtype == "bf16" else 1
+    w_gate_up = U * 2 * I * H * wb + S * 2 * Is * H * wb
+    w_down = U * H * I * wb + S * H * Is * wb
+    router = E * H * 4
+    x_read = valid_tokens * H * 2
+    out_write = w.T * H * 2
+    step_bytes = w_gate_up + w_down + router + x_read + out_write
+    expert_flops = 2 * routed_rows * 3 * H * I + 2 * valid_tokens * S * 3 * H * Is
+    router_flops = 2 * valid_tokens * E * H
+    rows = routed_rows + S * valid_tokens
+    gate_up_bytes = w_gate_up + rows * H * 2 + rows * max(I, Is) * 2
+    gate_up_flops = 2 * routed_rows * 2 * I * H + 2 * valid_tokens * S * 2 * Is * H
+    return {"touched_experts": U, "routed_rows": routed_rows, "step_bytes": step_bytes,
+            "step_flops": expert_flops + router_flops, "expert_flops": expert_flops,
+            "gate_up_bytes": gate_up_bytes, "gate_up_flops": gate_up_flops}
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3])
+                          if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_fp32_b200 as moe
+    from mixture_experts_fp32_b200 import build as lib_build
+    import synth
+
+    ws_n, rank, local = dist_env()
+    if ws_n > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        lib_build.build()
+    if ws_n > 1:
+        dist.barrier()
+    moe.load()
+
+    w = synth.WORKLOADS[args.workload]
+    k = w.k
+    # weights: drawn once (rank 0) and broadcast; activations: one batch per rank
+    inp = synth.make_inputs(w, with_weights=(rank == 0))
+    if ws_n > 1:
+        inp["x"] = synth.normal_bf16(w.seed + 1000 * rank, synth.STREAM_X, (w.T, w.H), w.x_sigma)
+    d = {}
+    for key in ("x", "valid", "router_w", "router_b"):
+        d[key] = None if inp.get(key) is None else inp[key].to(dev)
+    wkeys = ["w_gate_up", "w_down", "ws_gate_up", "ws_down", "s_gate_up", "s_down",
+             "ss_gate_up", "ss_down"]
+    for key in wkeys:
+        if rank == 0:
+            d[key] = None if inp.get(key) is None else inp[key].to(dev)
+    if ws_n > 1:
+        shapes = [None if d.get(kk) is None else (tuple(d[kk].shape), d[kk].dtype)
+                  for kk in wkeys] if rank == 0 else None
+        obj = [shapes]
+        dist.broadcast_object_list(obj, src=0)
+        shapes = obj[0]
+        for kk, sh in zip(wkeys, shapes):
+            if sh is None:
+                d[kk] = None
+                continue
+            if rank != 0:
+                d[kk] = torch.empty(sh[0], dtype=sh[1], device=dev)
+            dist.broadcast(d[kk], src=0)
+    del inp
+
+    plan = moe.Plan(max_tokens=w.T, hidden=w.H, num_experts=w.E, top_k_max=k, inter=w.I,
+                    num_shared=w.S, shared_inter=w.Is if w.S else 0, device=dev,
+                    wtype=moe.MOE_W_BF16 if w.wtype == "bf16" else moe.MOE_W_FP8_E4M3_B128)
+    weights = moe.make_weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
+                               d.get("s_gate_up"), d.get("s_down"), d.get("ws_gate_up"),
+                               d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    valid_tokens = int(d["valid"].sum().item())
+
+    def fwd(events=None, want_offsets=False):
+        dbg = moe.make_debug(offsets=offsets if want_offsets else None, events=events)
+        plan.forward(weights, d["x"], d["valid"], k, out, stream=stream, dbg=dbg)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        fwd(want_offsets=True)
+    torch.cuda.synchronize()
+    if plan.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    algo = algorithmic(w, valid_tokens, offsets.cpu().numpy(), k)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGES + 1)]
+          for _ in range(K)]
+    clocks = ClockSampler(dev.index)
+    if ws_n > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        flush.zero_()                      # L2 flush outside the step's events
+        fwd(events=ev[i])
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clock_info = clocks.stop()
+    if ws_n > 1:
+        dist.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][moe.MOE_NUM_STAGES]) for i in range(K)]
+    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(K))
+                for s, name in enumerate(moe.STAGE_NAMES)}
+    status = plan.device_status()
+    total_ms = sum(step_ms)
+    gemm_ms = stage_ms["gate_up_gemm"]
+
+    # end to end: pinned host input -> device, forward, result -> pinned host
+    x_host = d["x"].cpu().pin_memory()
+    v_host = d["valid"].cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    v_dev = torch.empty_like(d["valid"])
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        v_dev.copy_(v_host, non_blocking=True)
+        plan.forward(weights, x_dev, v_dev, k, out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(K):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        x_dev.copy_(x_host, non_blocking=True)
+        v_dev.copy_(v_host, non_blocking=True)
+        plan.forward(weights, x_dev, v_dev, k, out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+
+    def max_over_ranks(v: float) -> float:
+        if ws_n == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(v: float) -> float:
+        if ws_n == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    total_ms = max_over_ranks(total_ms)
+    e2e_total = max_over_ranks(sum(e2e_ms))
+    tokens = sum_over_ranks(float(valid_tokens))
+    gemm_ms_max = max_over_ranks(gemm_ms)
+    status = int(max_over_ranks(float(status)))
+
+    peaks = measured_peaks()
+    prefill = w.wtype == "fp8"
+    bound = "tensor" if prefill else "hbm"
+    if bound == "hbm":
+        achieved = algo["gate_up_bytes"] / (gemm_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = algo["gate_up_flops"] / (gemm_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"] * (2 if w.wtype == "fp8" else 1)
+        unit = "TFLOP/s"
+    ms = total_ms / K
+    step_roof_ms = max(algo["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                       algo["step_flops"] / (peaks["bf16_tflops"] * 1e12)) * 1e3
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(w, args) if (ws_n == 1 and not args.no_cpu_baseline) else None
+        result = {
+            "metric": METRIC, "value": tokens / (total_ms * 1e-3 / K) if K else 0.0,
+            "unit": "tokens/s", "n_gpus": ws_n, "steps": K, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.wtype, "data": "synthetic (Philox4x32-10, seed 0)",
+            "config": {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens, "H": w.H,
+                       "E": w.E, "k": k, "I": w.I, "S": w.S, "Is": w.Is,
+                       "parallelism": f"dp{ws_n} replicas" if ws_n > 1 else "single GPU",
+                       "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps, "
+                             "outside the step events; weights alone exceed L2"},
+            "roofline": {"bound": bound, "kernel": "grouped_gemm gate/up + SwiGLU",
+                         "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": peaks["source"]},
+            "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / ms,
+                              "algorithmic_bytes": algo["step_bytes"],
+                              "algorithmic_flops": algo["step_flops"],
+                              "touched_experts": algo["touched_experts"]},
+            "stage_ms": stage_ms,
+            "e2e": {"value": tokens / (e2e_total * 1e-3 / K), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_host.numel() * 2 + v_host.numel(),
+                    "d2h_bytes_per_step": out_host.numel() * 2},
+            "gpu_launches": 7 * K,
+            "clocks": clock_info,
+            "device_status": status,
+            "wall_s_timed_region": t_wall,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(result), flush=True)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+# --------------------------------------------------------- the CPU oracle
+
+def oracle_tokens_per_s(w, target_s: float):
+    """Times the oracle (routing and expert FFN) on growing samples of the
+    workload's valid tokens until one sample takes about target_s seconds."""
+    import numpy as np
+
+    import oracle
+    import synth
+    inp = synth.make_inputs(w)
+    valid_idx = np.nonzero(inp["valid"].numpy())[0]
+    cores = os.cpu_count() or 1
+    n = min(len(valid_idx), max(1, cores))
+    while True:
+        tok = valid_idx[:n]
+        t0 = time.perf_counter()
+        sub = dict(inp)
+        sub["x"] = inp["x"][tok]
+        sub["valid"] = inp["valid"][tok]
+        logits = oracle.router_logits(sub["x"], sub["valid"], inp["router_w"], inp["router_b"])
+        ids, wt = oracle.topk(logits, sub["valid"], w.k)
+        oracle.route(ids, sub["valid"], w.E)
+        oracle.moe_tokens(sub, ids, wt)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or n >= len(valid_idx):
+            return n / dt, n, dt, cores
+        n = min(len(valid_idx), int(n * max(2.0, target_s / max(dt, 1e-3))))
+
+
+def cpu_baseline(w, args):
+    rate, n, dt, cores = oracle_tokens_per_s(w, args.cpu_seconds)
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} valid tokens of {w.name} (all weights), {dt:.1f} s, "
+                      f"double-precision C with OpenMP over tokens"}
+
+
+def run_reference(args):
+    ws_n, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    rates = []
+    for _ in range(max(args.warmup, 0)):
+        oracle_tokens_per_s(w, min(args.cpu_seconds, 5.0))
+    n = dt = cores = 0
+    for _ in range(args.steps):
+        r, n, dt, cores = oracle_tokens_per_s(w, args.cpu_seconds)
+        rates.append(r)
+    value = statistics.median(rates) if rates else 0.0
+    res = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * n / value if value else 0,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (Philox4x32-10, seed 0)", "impl": "reference",
+           "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k, "I": w.I,
+                      "S": w.S, "Is": w.Is},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle",
+                            "sample": f"{n} valid tokens per step of {w.name}, {dt:.1f} s"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+    return res
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+/*
+ * moe.h — C ABI of a B200 (sm_100a) library for the forward pass of one
+ * Mixture-of-Experts layer.
+ *
+ * The layer (Step3 推論最適化 (MI308X vs H20), §背景: "3-in-48" expert
+ * selection; §最適化技術: one-stage MoE kernel tuned along inter_dim, shared
+ * expert MLP fused into the layer, mixed BF16 / FP8 block-scale GEMMs;
+ * [SGLang] MoE 모델을 위한 Single Batch Overlap 기법, §들어가며: dispatch,
+ * down projection GEMM, combine) computes, for every valid row t of x:
+ *
+ *   l[t,e]   = sum_h x[t,h] Wr[e,h] (+ b[e])                 router logits (fp32)
+ *   ids[t,:] = the k largest l[t,e], descending, ties to the lower e
+ *   w[t,j]   = exp(l[t,ids_j] - l[t,ids_0]) / sum_j' exp(...)   (renormalised)
+ *              or the full-softmax probability of ids_j (renormalize = 0)
+ *   y_e(x)   = Wd[e] (silu(Wg[e] x) * (Wu[e] x)),  silu(z) = z / (1 + e^-z)
+ *   out[t]   = bf16( sum_j w[t,j] y_{ids_j}(x[t]) + y_shared(x[t]) )
+ *
+ * and writes +0.0 to every row whose valid flag is 0 (padding rows of a
+ * data-parallel all_gather, DP Attention and TBO for DeepSeek-V4 on MI355X,
+ * §PrefillDelayer): such rows are not routed and not computed, and their
+ * contents never matter.
+ *
+ * Conventions for every entry point:
+ *  - All tensors are dense and row-major.  Device pointers are addresses in
+ *    the current CUDA device's memory, owned by the caller; the library never
+ *    allocates, frees or retains device memory.  Host pointers are read only
+ *    during the call.
+ *  - Device pointers to tensors must be 16-byte aligned; the workspace must be
+ *    256-byte aligned.
+ *  - Work is enqueued on the given cudaStream_t (passed as void*, NULL = the
+ *    legacy default stream) without host synchronisation, device-to-host
+ *    copies or allocation, so moe_forward can be captured in a CUDA graph once
+ *    it has been called on the device outside capture (the first call sets
+ *    kernel attributes).
+ *  - Argument errors are detected on the host before anything is enqueued and
+ *    return a negative moe_status; nothing is launched in that case.
+ *  - Failures detected on the device (a bounded wait that expired, an expert
+ *    index out of range) set bits in a status word inside the workspace; read
+ *    them with moe_check_device_status.  The library never aborts the process
+ *    and never traps on the device.
+ *  - One workspace may serve one forward at a time: calls that share a
+ *    workspace must be ordered on one stream.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,   /* a null pointer, a size out of range, misalignment */
+    MOE_ERR_UNSUPPORTED = -2,   /* a shape or type this build does not implement */
+    MOE_ERR_WORKSPACE = -3,     /* workspace smaller than moe_plan_create reported */
+    MOE_ERR_CUDA = -4,          /* a CUDA runtime call failed (launch, attribute, sync) */
+    MOE_ERR_DEVICE = -5         /* moe_check_device_status found a device-side failure */
+} moe_status;
+
+typedef enum {
+    MOE_W_BF16 = 0,             /* bf16 expert weights */
+    MOE_W_FP8_E4M3_B128 = 1     /* OCP e4m3 weights with one fp32 scale per 128x128 block;
+                                   activations quantised e4m3 per 1x128 group inside the call */
+} moe_wtype;
+
+/* Device status bits (moe_check_device_status). */
+#define MOE_DEV_WAIT_TIMEOUT_GATE_UP 0x1u   /* a bounded wait expired in the gate/up GEMM */
+#define MOE_DEV_WAIT_TIMEOUT_DOWN    0x2u   /* a bounded wait expired in the down GEMM */
+#define MOE_DEV_BAD_EXPERT_ID        0x4u   /* a routed expert index outside [0, E) */
+
+/* Shape of the layer; fixed for the lifetime of a plan. */
+typedef struct {
+    int max_tokens;     /* largest T a forward will be given (rows, valid + padding), >= 1 */
+    int hidden;         /* H: multiple of 128 */
+    int num_experts;    /* E: 1..256 routed experts */
+    int top_k_max;      /* largest k a forward will be given: 1..min(8, E) */
+    int inter;          /* I: routed expert intermediate size, multiple of 128 */
+    int num_shared;     /* S: 0 or 1 always-on shared expert */
+    int shared_inter;   /* Is: shared expert intermediate size, multiple of 128 (S = 1) */
+    int renormalize;    /* 1: softmax over the selected k; 0: full softmax over E */
+    moe_wtype wtype;
+} moe_config;
+
+typedef struct moe_plan_s *moe_plan_t;
+
+/* Validates the shape and sizes the workspace.  Host only: touches no device.
+ * *plan receives a new plan (free with moe_plan_destroy), *workspace_bytes the
+ * device workspace size every forward with this plan needs. */
+moe_status moe_plan_create(const moe_config *cfg, moe_plan_t *plan, size_t *workspace_bytes);
+void moe_plan_destroy(moe_plan_t plan);
+
+/* Upper bound on every device-side wait, in nanoseconds (default 2e9).  A
+ * wait that runs out sets a MOE_DEV_WAIT_TIMEOUT_* bit and its kernel returns
+ * early with its output incomplete.  0 makes every wait that is not already
+ * satisfied give up at once; it exists to exercise that path. */
+moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns);
+
+/* Weights (device pointers).
+ *  router_w   fp32 [E, H];  router_b fp32 [E] or NULL (added to the logits)
+ *  w_gate_up  [E, 2I, H]: rows 0..I-1 of each expert are the gate projection,
+ *             rows I..2I-1 the up projection (bf16, or e4m3 codes as bytes)
+ *  w_down     [E, H, I]
+ *  s_gate_up  fp32 [E, 2I/128, H/128], s_down fp32 [E, H/128, I/128] (FP8 only)
+ *  ws_gate_up [2Is, H], ws_down [H, Is], ss_* likewise: the shared expert
+ *             (NULL when num_shared = 0). */
+typedef struct {
+    const float *router_w;
+    const float *router_b;
+    const void *w_gate_up;
+    const void *w_down;
+    const float *s_gate_up;
+    const float *s_down;
+    const void *ws_gate_up;
+    const void *ws_down;
+    const float *ss_gate_up;
+    const float *ss_down;
+} moe_weights;
+
+/* Optional copies of intermediate results (device pointers, each may be NULL):
+ *  logits    fp32 [T, E]   (0 in padding rows)
+ *  topk_ids  int32 [T, k]  (-1 in padding rows)
+ *  topk_w    fp32 [T, k]   (0 in padding rows)
+ *  perm      int32 [T*k]   first Tv*k entries: pair index t*k+j, grouped by
+ *                          expert, ascending t inside an expert
+ *  offsets   int32 [E+1]   exclusive prefix sum of the per-expert pair counts
+ *  events    cudaEvent_t handles (as void*) recorded on the stream before the
+ *            first stage and after each of the MOE_NUM_STAGES stages
+ *            (router, top-k, permute, gather, gate/up GEMM, down GEMM,
+ *            combine); NULL entries are skipped. */
+#define MOE_NUM_STAGES 7
+typedef struct {
+    float *logits;
+    int *topk_ids;
+    float *topk_w;
+    int *perm;
+    int *offsets;
+    void *events[MOE_NUM_STAGES + 1];
+} moe_debug;
+
+/* The forward pass.
+ *  hidden  bf16 [T, H] (device);  valid uint8 [T] (device; NULL = all rows valid)
+ *  T       0..max_tokens rows;  k  1..top_k_max experts per token
+ *  out     bf16 [T, H] (device), fully written (padding rows get +0.0)
+ *  workspace / ws_bytes: device scratch of at least the size moe_plan_create gave
+ *  stream  cudaStream_t;  dbg  optional, may be NULL. */
+moe_status moe_forward(moe_plan_t plan, const moe_weights *weights, const void *hidden,
+                       const uint8_t *valid, int T, int k, void *out, void *workspace,
+                       size_t ws_bytes, void *stream, moe_debug *dbg);
+
+/* Routing only, from given fp32 logits [T, E] (device): the top-k selection,
+ * weights, per-expert offsets and permutation exactly as moe_forward computes
+ * them.  Outputs as in moe_debug (topk_ids, topk_w [T,k]; perm [T*k];
+ * offsets [E+1]); none may be NULL. */
+moe_status moe_route_from_logits(moe_plan_t plan, const float *logits, const uint8_t *valid,
+                                 int T, int k, int *topk_ids, float *topk_w, int *perm,
+                                 int *offsets, void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronises the stream, reads and clears the device status word of this
+ * workspace.  *bits (may be NULL) receives the MOE_DEV_* bits that were set.
+ * Returns MOE_OK if none, MOE_ERR_DEVICE otherwise. */
+moe_status moe_check_device_status(moe_plan_t plan, void *workspace, void *stream,
+                                   uint32_t *bits);
+
+/* Device addresses of the intermediate buffers inside a workspace, for
+ * inspection after a forward (host arithmetic only; nothing is launched):
+ *  row_token  int32 [R]     token index of each permuted row (R = Tv*(k+S))
+ *  x_perm     [R, H]        permuted activations (bf16; e4m3 codes for FP8)
+ *  h          [R, Imax]     SwiGLU output rows (bf16; e4m3 codes for FP8)
+ *  y          bf16 [R, H]   expert output rows before the weighted combine
+ *  group_offsets int32 [E+S+1]: rows of expert e are [go[e], go[e+1]); the
+ *             shared expert is group E. */
+typedef struct {
+    int *row_token;
+    void *x_perm;
+    void *h;
+    void *y;
+    int *group_offsets;
+    int h_stride;       /* Imax = max(I, Is) elements per h row */
+} moe_workspace_views;
+moe_status moe_get_workspace_views(moe_plan_t plan, void *workspace, moe_workspace_views *views);
+
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,236 @@
+"""Python binding of the B200 MoE-layer library (include/moe.h).
+
+Argument marshalling only: every function here forwards to the C ABI entry
+point of the same name in libmoe_b200.so, passing torch tensors' device
+addresses.  There is no fallback: if the library is missing or a call fails,
+an exception is raised.  PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_WORKSPACE = -3
+MOE_ERR_CUDA = -4
+MOE_ERR_DEVICE = -5
+
+MOE_W_BF16 = 0
+MOE_W_FP8_E4M3_B128 = 1
+
+MOE_DEV_WAIT_TIMEOUT_GATE_UP = 0x1
+MOE_DEV_WAIT_TIMEOUT_DOWN = 0x2
+MOE_DEV_BAD_EXPERT_ID = 0x4
+
+MOE_NUM_STAGES = 7
+STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")
+
+EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
+            "moe_route_from_logits", "moe_check_device_status", "moe_get_workspace_views",
+            "moe_status_string")
+
+_c_int = ctypes.c_int
+_vp = ctypes.c_void_p
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("max_tokens", _c_int), ("hidden", _c_int), ("num_experts", _c_int),
+                ("top_k_max", _c_int), ("inter", _c_int), ("num_shared", _c_int),
+                ("shared_inter", _c_int), ("renormalize", _c_int), ("wtype", _c_int)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [("router_w", _vp), ("router_b", _vp), ("w_gate_up", _vp), ("w_down", _vp),
+                ("s_gate_up", _vp), ("s_down", _vp), ("ws_gate_up", _vp), ("ws_down", _vp),
+                ("ss_gate_up", _vp), ("ss_down", _vp)]
+
+
+class moe_debug(ctypes.Structure):
+    _fields_ = [("logits", _vp), ("topk_ids", _vp), ("topk_w", _vp), ("perm", _vp),
+                ("offsets", _vp), ("events", _vp * (MOE_NUM_STAGES + 1))]
+
+
+class moe_workspace_views(ctypes.Structure):
+    _fields_ = [("row_token", _vp), ("x_perm", _vp), ("h", _vp), ("y", _vp),
+                ("group_offsets", _vp), ("h_stride", _c_int)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def load():
+    """Loads libmoe_b200.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: run mixture_experts_fp32_b200.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    L.moe_plan_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(_vp),
+                                  ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_plan_create.restype = _c_int
+    L.moe_plan_destroy.argtypes = [_vp]
+    L.moe_plan_destroy.restype = None
+    L.moe_plan_set_wait_limit.argtypes = [_vp, ctypes.c_uint64]
+    L.moe_plan_set_wait_limit.restype = _c_int
+    L.moe_forward.argtypes = [_vp, ctypes.POINTER(moe_weights), _vp, _vp, _c_int, _c_int, _vp, _vp,
+                              ctypes.c_size_t, _vp, ctypes.POINTER(moe_debug)]
+    L.moe_forward.restype = _c_int
+    L.moe_route_from_logits.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
+                                        ctypes.c_size_t, _vp]
+    L.moe_route_from_logits.restype = _c_int
+    L.moe_check_device_status.argtypes = [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.moe_check_device_status.restype = _c_int
+    L.moe_get_workspace_views.argtypes = [_vp, _vp, ctypes.POINTER(moe_workspace_views)]
+    L.moe_get_workspace_views.restype = _c_int
+    L.moe_status_string.argtypes = [_c_int]
+    L.moe_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _addr(t) -> int | None:
+    """Device (or host) address of a tensor, an int address, or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def moe_status_string(status: int) -> str:
+    return load().moe_status_string(status).decode()
+
+
+def moe_plan_create(cfg: moe_config):
+    """Returns (plan handle, workspace bytes)."""
+    plan = _vp()
+    ws = ctypes.c_size_t()
+    _check(load().moe_plan_create(ctypes.byref(cfg), ctypes.byref(plan), ctypes.byref(ws)),
+           "moe_plan_create")
+    return plan.value, ws.value
+
+
+def moe_plan_destroy(plan) -> None:
+    load().moe_plan_destroy(plan)
+
+
+def moe_plan_set_wait_limit(plan, limit_ns: int) -> None:
+    _check(load().moe_plan_set_wait_limit(plan, limit_ns), "moe_plan_set_wait_limit")
+
+
+def make_weights(router_w, router_b=None, w_gate_up=None, w_down=None, s_gate_up=None,
+                 s_down=None, ws_gate_up=None, ws_down=None, ss_gate_up=None,
+                 ss_down=None) -> moe_weights:
+    return moe_weights(*[_addr(t) for t in (router_w, router_b, w_gate_up, w_down, s_gate_up,
+                                             s_down, ws_gate_up, ws_down, ss_gate_up, ss_down)])
+
+
+def make_debug(logits=None, topk_ids=None, topk_w=None, perm=None, offsets=None,
+               events=None) -> moe_debug:
+    d = moe_debug(_addr(logits), _addr(topk_ids), _addr(topk_w), _addr(perm), _addr(offsets))
+    if events is not None:
+        for i, ev in enumerate(events):
+            d.events[i] = None if ev is None else ev.cuda_event
+    return d
+
+
+def moe_forward(plan, weights: moe_weights, hidden, valid, T: int, k: int, out, workspace,
+                ws_bytes: int, stream=None, dbg: moe_debug | None = None) -> None:
+    st = load().moe_forward(plan, ctypes.byref(weights), _addr(hidden), _addr(valid), T, k,
+                            _addr(out), _addr(workspace), ws_bytes, _stream(stream),
+                            None if dbg is None else ctypes.byref(dbg))
+    _check(st, "moe_forward")
+
+
+def moe_route_from_logits(plan, logits, valid, T: int, k: int, topk_ids, topk_w, perm, offsets,
+                          workspace, ws_bytes: int, stream=None) -> None:
+    st = load().moe_route_from_logits(plan, _addr(logits), _addr(valid), T, k, _addr(topk_ids),
+                                      _addr(topk_w), _addr(perm), _addr(offsets),
+                                      _addr(workspace), ws_bytes, _stream(stream))
+    _check(st, "moe_route_from_logits")
+
+
+def moe_check_device_status(plan, workspace, stream=None) -> int:
+    """Returns the device status bits (0 = none); synchronises the stream."""
+    bits = ctypes.c_uint32()
+    st = load().moe_check_device_status(plan, _addr(workspace), _stream(stream),
+                                        ctypes.byref(bits))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoeError(st, "moe_check_device_status")
+    return bits.value
+
+
+def moe_get_workspace_views(plan, workspace) -> moe_workspace_views:
+    v = moe_workspace_views()
+    _check(load().moe_get_workspace_views(plan, _addr(workspace), ctypes.byref(v)),
+           "moe_get_workspace_views")
+    return v
+
+
+class Plan:
+    """A plan plus a torch-allocated workspace on the current device."""
+
+    def __init__(self, *, max_tokens: int, hidden: int, num_experts: int, top_k_max: int,
+                 inter: int, num_shared: int = 0, shared_inter: int = 0, renormalize: int = 1,
+                 wtype: int = MOE_W_BF16, device=None):
+        import torch
+        self.cfg = moe_config(max_tokens, hidden, num_experts, top_k_max, inter, num_shared,
+                              shared_inter, renormalize, wtype)
+        self.handle, self.ws_bytes = moe_plan_create(self.cfg)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8,
+                                     device=device if device is not None else "cuda")
+
+    def forward(self, weights: moe_weights, hidden, valid, k: int, out, stream=None, dbg=None):
+        moe_forward(self.handle, weights, hidden, valid, hidden.shape[0], k, out, self.workspace,
+                    self.ws_bytes, stream, dbg)
+
+    def route_from_logits(self, logits, valid, k: int, topk_ids, topk_w, perm, offsets,
+                          stream=None):
+        moe_route_from_logits(self.handle, logits, valid, logits.shape[0], k, topk_ids, topk_w,
+                              perm, offsets, self.workspace, self.ws_bytes, stream)
+
+    def device_status(self, stream=None) -> int:
+        return moe_check_device_status(self.handle, self.workspace, stream)
+
+    def views(self) -> moe_workspace_views:
+        return moe_get_workspace_views(self.handle, self.workspace)
+
+    def set_wait_limit(self, ns: int):
+        moe_plan_set_wait_limit(self.handle, ns)
+
+    def close(self):
+        if self.handle:
+            moe_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

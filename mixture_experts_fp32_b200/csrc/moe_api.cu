@@ -1,0 +1,341 @@
+// The C ABI declared in include/moe.h: plan (shape validation, workspace
+// layout), argument checks, and the launch sequence of one MoE-layer forward
+// pass on one stream.  No allocation, no host synchronisation, no
+// device-to-host copy on the forward path.
+#include <string.h>
+
+#include <new>
+
+#include "moe_internal.cuh"
+
+#define MOE_EXPORT extern "C" __attribute__((visibility("default")))
+
+struct moe_plan_s {
+  moe_config cfg;
+  size_t ws_bytes;
+  int imax;          // max(I, Is)
+  int ks_max;        // top_k_max + S
+  size_t r_cap;      // max_tokens * ks_max rows
+  // byte offsets inside the workspace
+  size_t off_status, off_goff, off_partial, off_logits, off_ids, off_w, off_perm, off_inv,
+      off_rowtok, off_xp, off_h, off_y;
+  unsigned long long wait_limit_ns;
+  int device;
+  int num_sms;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status ensure_device(moe_plan_s* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (p->device == dev) return MOE_OK;
+  static unsigned long long prepared_mask = 0;   // devices whose kernel attributes are set
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
+  if (dev < 64 && !((prepared_mask >> dev) & 1ull)) {
+    if (moe::prepare_grouped_gemm_kernels() != cudaSuccess) return MOE_ERR_CUDA;
+    prepared_mask |= 1ull << dev;
+  }
+  p->num_sms = sms;
+  p->device = dev;
+  return MOE_OK;
+}
+
+moe_status check_launch(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+void record(moe_debug* dbg, int i, cudaStream_t st) {
+  if (dbg != nullptr && dbg->events[i] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(dbg->events[i]), st);
+}
+
+moe_status check_common(const moe_plan_s* p, int T, int k, const void* workspace,
+                        size_t ws_bytes) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > p->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > p->cfg.top_k_max) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < p->ws_bytes) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_EXPORT const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape, type or device";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE: return "device-side failure (see status bits)";
+  }
+  return "unknown status";
+}
+
+MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
+                                      size_t* workspace_bytes) {
+  if (cfg == nullptr || plan == nullptr || workspace_bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *plan = nullptr;
+  const moe_config c = *cfg;
+  if (c.max_tokens < 1 || c.hidden < 1 || c.num_experts < 1 || c.top_k_max < 1 || c.inter < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (c.num_shared != 0 && c.num_shared != 1) return MOE_ERR_INVALID_ARG;
+  if (c.renormalize != 0 && c.renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (c.wtype != MOE_W_BF16 && c.wtype != MOE_W_FP8_E4M3_B128) return MOE_ERR_INVALID_ARG;
+  if (c.top_k_max > c.num_experts) return MOE_ERR_INVALID_ARG;
+  if (c.num_shared == 1 && c.shared_inter < 1) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts > moe::kMaxExperts || c.top_k_max > moe::kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (c.hidden % 128 != 0 || c.inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c.num_shared == 1 && c.shared_inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c.hidden > 65536 || c.inter > 65536 || c.shared_inter > 65536) return MOE_ERR_UNSUPPORTED;
+  if (c.wtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;   // e4m3 block-scale path not built yet
+  const int S = c.num_shared;
+  const int imax = S && c.shared_inter > c.inter ? c.shared_inter : c.inter;
+  const size_t T = (size_t)c.max_tokens, E = (size_t)c.num_experts, H = (size_t)c.hidden;
+  const size_t ks = (size_t)c.top_k_max + S;
+  const size_t r_cap = T * ks;
+  if (r_cap > (size_t)0x7fffffff / 2) return MOE_ERR_UNSUPPORTED;
+
+  moe_plan_s* p = new (std::nothrow) moe_plan_s();
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  p->cfg = c;
+  p->imax = imax;
+  p->ks_max = (int)ks;
+  p->r_cap = r_cap;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  p->off_status = take(64);
+  p->off_goff = take(sizeof(int) * (E + 2));
+  p->off_partial = take(sizeof(float) * moe::kRouterSplitMax * T * E);
+  p->off_logits = take(sizeof(float) * T * E);
+  p->off_ids = take(sizeof(int) * T * c.top_k_max);
+  p->off_w = take(sizeof(float) * T * c.top_k_max);
+  p->off_perm = take(sizeof(int) * T * c.top_k_max);
+  p->off_inv = take(sizeof(int) * T * ks);
+  p->off_rowtok = take(sizeof(int) * r_cap);
+  p->off_xp = take(2 * r_cap * H);
+  p->off_h = take(2 * r_cap * (size_t)imax);
+  p->off_y = take(2 * r_cap * H);
+  p->ws_bytes = off;
+  p->wait_limit_ns = 2000000000ull;
+  p->device = -1;
+  p->num_sms = 0;
+  *plan = p;
+  *workspace_bytes = p->ws_bytes;
+  return MOE_OK;
+}
+
+MOE_EXPORT void moe_plan_destroy(moe_plan_t plan) { delete plan; }
+
+MOE_EXPORT moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  plan->wait_limit_ns = limit_ns;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const void* hidden,
+                                  const uint8_t* valid, int T, int k, void* out, void* workspace,
+                                  size_t ws_bytes, void* stream, moe_debug* dbg) {
+  moe_status s = check_common(plan, T, k, workspace, ws_bytes);
+  if (s != MOE_OK) return s;
+  if (wts == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  const moe_config& c = plan->cfg;
+  const int S = c.num_shared;
+  if (hidden == nullptr || out == nullptr || wts->router_w == nullptr ||
+      wts->w_gate_up == nullptr || wts->w_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (S && (wts->ws_gate_up == nullptr || wts->ws_down == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(out) || !aligned16(wts->router_w) ||
+      !aligned16(wts->w_gate_up) || !aligned16(wts->w_down) ||
+      (S && (!aligned16(wts->ws_gate_up) || !aligned16(wts->ws_down))))
+    return MOE_ERR_INVALID_ARG;
+  if ((wts->router_b != nullptr && (reinterpret_cast<uintptr_t>(wts->router_b) & 3u)) != 0)
+    return MOE_ERR_INVALID_ARG;
+  s = ensure_device(plan);
+  if (s != MOE_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = c.num_experts, H = c.hidden, I = c.inter, Is = S ? c.shared_inter : 0;
+  const int G = E + S;
+  const int ks = k + S;
+  const int R_cap = T * ks;
+  unsigned int* status = at<unsigned int>(workspace, plan->off_status);
+  int* goff = at<int>(workspace, plan->off_goff);
+  float* partial = at<float>(workspace, plan->off_partial);
+  float* logits = at<float>(workspace, plan->off_logits);
+  int* ids = at<int>(workspace, plan->off_ids);
+  float* w = at<float>(workspace, plan->off_w);
+  int* perm = at<int>(workspace, plan->off_perm);
+  int* inv = at<int>(workspace, plan->off_inv);
+  int* rowtok = at<int>(workspace, plan->off_rowtok);
+  auto* xp = at<__nv_bfloat16>(workspace, plan->off_xp);
+  auto* h = at<__nv_bfloat16>(workspace, plan->off_h);
+  auto* y = at<__nv_bfloat16>(workspace, plan->off_y);
+  const auto* x = static_cast<const __nv_bfloat16*>(hidden);
+
+  record(dbg, 0, st);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
+  int splits = 1, kchunk = H;
+  moe::router_split_plan(T, E, H, plan->num_sms, &splits, &kchunk);
+  s = check_launch(moe::launch_router_logits(x, valid, T, H, wts->router_w, E, partial, splits,
+                                             kchunk, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 1, st);
+  s = check_launch(moe::launch_topk(partial, splits, wts->router_b, valid, T, E, k, c.renormalize,
+                                    logits, ids, w, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 2, st);
+  s = check_launch(moe::launch_route(ids, valid, T, E, k, S, goff, perm, inv, rowtok, status, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 3, st);
+  s = check_launch(moe::launch_gather_rows(x, H, rowtok, goff + G, R_cap, xp, plan->num_sms, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 4, st);
+
+  moe::GroupedGemmArgs ga;
+  memset(&ga, 0, sizeof(ga));
+  ga.a_routed = wts->w_gate_up;
+  ga.a_shared = S ? wts->ws_gate_up : nullptr;
+  ga.b = xp;
+  ga.d = h;
+  ga.group_offsets = goff;
+  ga.E = E;
+  ga.G = G;
+  ga.K_routed = H;
+  ga.K_shared = H;
+  ga.K_ld = H;
+  ga.rows_per_expert = 2 * I;
+  ga.m_tiles_routed = I / 128;
+  ga.m_tiles_shared = S ? Is / 128 : 0;
+  ga.up_routed = I;
+  ga.up_shared = Is;
+  ga.ldd = plan->imax;
+  ga.R_cap = R_cap;
+  ga.gated = true;
+  ga.status = status;
+  ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_GATE_UP;
+  ga.wait_limit_ns = plan->wait_limit_ns;
+  ga.num_ctas = plan->num_sms;
+  s = check_launch(moe::launch_grouped_gemm(ga, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 5, st);
+
+  ga.a_routed = wts->w_down;
+  ga.a_shared = S ? wts->ws_down : nullptr;
+  ga.b = h;
+  ga.d = y;
+  ga.K_routed = I;
+  ga.K_shared = S ? Is : 0;
+  ga.K_ld = plan->imax;
+  ga.rows_per_expert = H;
+  ga.m_tiles_routed = H / 128;
+  ga.m_tiles_shared = S ? H / 128 : 0;
+  ga.up_routed = 0;
+  ga.up_shared = 0;
+  ga.ldd = H;
+  ga.gated = false;
+  ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
+  s = check_launch(moe::launch_grouped_gemm(ga, st));
+  if (s != MOE_OK) return s;
+  record(dbg, 6, st);
+
+  s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S,
+                                       static_cast<__nv_bfloat16*>(out), st));
+  if (s != MOE_OK) return s;
+  record(dbg, 7, st);
+
+  if (dbg != nullptr) {
+    const auto d2d = cudaMemcpyDeviceToDevice;
+    if (dbg->logits && cudaMemcpyAsync(dbg->logits, logits, sizeof(float) * T * E, d2d, st))
+      return MOE_ERR_CUDA;
+    if (dbg->topk_ids && cudaMemcpyAsync(dbg->topk_ids, ids, sizeof(int) * T * k, d2d, st))
+      return MOE_ERR_CUDA;
+    if (dbg->topk_w && cudaMemcpyAsync(dbg->topk_w, w, sizeof(float) * T * k, d2d, st))
+      return MOE_ERR_CUDA;
+    if (dbg->perm && cudaMemcpyAsync(dbg->perm, perm, sizeof(int) * T * k, d2d, st))
+      return MOE_ERR_CUDA;
+    if (dbg->offsets && cudaMemcpyAsync(dbg->offsets, goff, sizeof(int) * (E + 1), d2d, st))
+      return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_route_from_logits(moe_plan_t plan, const float* logits,
+                                            const uint8_t* valid, int T, int k, int* topk_ids,
+                                            float* topk_w, int* perm, int* offsets,
+                                            void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_common(plan, T, k, workspace, ws_bytes);
+  if (s != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr || perm == nullptr ||
+      offsets == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  s = ensure_device(plan);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const moe_config& c = plan->cfg;
+  const int E = c.num_experts, S = c.num_shared;
+  unsigned int* status = at<unsigned int>(workspace, plan->off_status);
+  int* goff = at<int>(workspace, plan->off_goff);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
+  s = check_launch(moe::launch_topk(logits, 1, nullptr, valid, T, E, k, c.renormalize,
+                                    at<float>(workspace, plan->off_logits), topk_ids, topk_w, st));
+  if (s != MOE_OK) return s;
+  s = check_launch(moe::launch_route(topk_ids, valid, T, E, k, S, goff, perm,
+                                     at<int>(workspace, plan->off_inv),
+                                     at<int>(workspace, plan->off_rowtok), status, st));
+  if (s != MOE_OK) return s;
+  if (cudaMemcpyAsync(offsets, goff, sizeof(int) * (E + 1), cudaMemcpyDeviceToDevice, st) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_check_device_status(moe_plan_t plan, void* workspace, void* stream,
+                                              uint32_t* bits) {
+  if (plan == nullptr || workspace == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = at<unsigned int>(workspace, plan->off_status);
+  unsigned int v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemset(status, 0, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (bits != nullptr) *bits = v;
+  return v == 0 ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+MOE_EXPORT moe_status moe_get_workspace_views(moe_plan_t plan, void* workspace,
+                                              moe_workspace_views* v) {
+  if (plan == nullptr || workspace == nullptr || v == nullptr) return MOE_ERR_INVALID_ARG;
+  v->row_token = at<int>(workspace, plan->off_rowtok);
+  v->x_perm = at<void>(workspace, plan->off_xp);
+  v->h = at<void>(workspace, plan->off_h);
+  v->y = at<void>(workspace, plan->off_y);
+  v->group_offsets = at<int>(workspace, plan->off_goff);
+  v->h_stride = plan->imax;
+  return MOE_OK;
+}

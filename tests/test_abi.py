@@ -1,0 +1,128 @@
+"""The C ABI without a GPU: the library builds and loads, exports every entry
+point include/moe.h declares, and rejects bad arguments on the host before
+anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_fp32_b200 as moe
+from mixture_experts_fp32_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(moe.EXPORTED)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", moe.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+    # nothing else with C linkage leaks out under the moe_ prefix
+    assert {e for e in exported if e.startswith("moe_")} == set(names)
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.check_output(["cuobjdump", "--list-elf", moe.LIB_PATH], text=True)
+    assert "sm_100a" in out
+
+
+def cfg(**kw):
+    base = dict(max_tokens=256, hidden=7168, num_experts=48, top_k_max=3, inter=5120,
+                num_shared=1, shared_inter=5120, renormalize=1, wtype=moe.MOE_W_BF16)
+    base.update(kw)
+    return moe.moe_config(**base)
+
+
+def test_plan_create_and_workspace_size(lib):
+    plan, ws = moe.moe_plan_create(cfg())
+    try:
+        assert ws > 0 and ws % 256 == 0
+        T, H, E, k, I, S = 256, 7168, 48, 3, 5120, 1
+        R = T * (k + S)
+        at_least = 2 * R * H * 2 + 2 * R * I + 4 * T * E
+        assert ws >= at_least
+        v = moe.moe_get_workspace_views(plan, 1 << 20)
+        assert v.h_stride == I
+        assert v.row_token is not None and v.row_token > (1 << 20)
+    finally:
+        moe.moe_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(max_tokens=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(hidden=7000), moe.MOE_ERR_UNSUPPORTED),
+    (dict(inter=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(num_experts=257, top_k_max=3), moe.MOE_ERR_UNSUPPORTED),
+    (dict(top_k_max=9, num_experts=48), moe.MOE_ERR_UNSUPPORTED),
+    (dict(top_k_max=5, num_experts=4), moe.MOE_ERR_INVALID_ARG),
+    (dict(num_shared=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(num_shared=1, shared_inter=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(num_shared=1, shared_inter=200), moe.MOE_ERR_UNSUPPORTED),
+    (dict(renormalize=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(wtype=7), moe.MOE_ERR_INVALID_ARG),
+])
+def test_plan_create_rejects(lib, bad, status):
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_plan_create(cfg(**bad))
+    assert ei.value.status == status
+
+
+def test_null_arguments(lib):
+    plan = ctypes.c_void_p()
+    ws = ctypes.c_size_t()
+    assert lib.moe_plan_create(None, ctypes.byref(plan), ctypes.byref(ws)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_plan_set_wait_limit(None, 0) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(None, None, None, None, 1, 1, None, None, 0, None, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    for s in (0, -1, -2, -3, -4, -5):
+        assert moe.moe_status_string(s)
+
+
+def test_forward_rejects_bad_arguments_before_launch(lib):
+    # every case below must fail on the host: no CUDA device exists here
+    plan, ws = moe.moe_plan_create(cfg())
+    try:
+        w = moe.make_weights(0x1000, None, 0x2000, 0x3000, ws_gate_up=0x4000, ws_down=0x5000)
+        WS = 0x100000
+        good = dict(hidden=0x6000, valid=None, T=16, k=3, out=0x7000, workspace=WS, ws_bytes=ws)
+
+        def call(**kw):
+            a = dict(good)
+            a.update(kw)
+            return lib.moe_forward(plan, ctypes.byref(w), a["hidden"], a["valid"], a["T"], a["k"],
+                                   a["out"], a["workspace"], a["ws_bytes"], None, None)
+
+        assert call(T=257) == moe.MOE_ERR_INVALID_ARG          # T > max_tokens
+        assert call(T=-1) == moe.MOE_ERR_INVALID_ARG
+        assert call(k=0) == moe.MOE_ERR_INVALID_ARG
+        assert call(k=4) == moe.MOE_ERR_INVALID_ARG            # k > top_k_max
+        assert call(ws_bytes=ws - 1) == moe.MOE_ERR_WORKSPACE
+        assert call(workspace=WS + 16) == moe.MOE_ERR_INVALID_ARG   # not 256-byte aligned
+        assert call(workspace=None) == moe.MOE_ERR_INVALID_ARG
+        assert call(hidden=None) == moe.MOE_ERR_INVALID_ARG
+        assert call(out=0x7008) == moe.MOE_ERR_INVALID_ARG     # not 16-byte aligned
+        assert call(T=0) == moe.MOE_OK                          # nothing to do, nothing launched
+        w_noshared = moe.make_weights(0x1000, None, 0x2000, 0x3000)
+        assert lib.moe_forward(plan, ctypes.byref(w_noshared), 0x6000, None, 16, 3, 0x7000, WS,
+                               ws, None, None) == moe.MOE_ERR_INVALID_ARG
+        assert lib.moe_route_from_logits(plan, None, None, 4, 3, 0x10, 0x20, 0x30, 0x40, WS, ws,
+                                         None) == moe.MOE_ERR_INVALID_ARG
+    finally:
+        moe.moe_plan_destroy(plan)
