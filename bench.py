@@ -206,6 +206,11 @@ def run_native(args):
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGES + 1)]
           for _ in range(K)]
+    # torch creates the CUDA event on first record; the library records them again in-step
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
     clocks = ClockSampler(dev.index)
     if ws_n > 1:
         dist.barrier()

@@ -169,7 +169,7 @@ moe_status moe_check_device_status(moe_plan_t plan, void *workspace, void *strea
  *  row_token  int32 [R]     token index of each permuted row (R = Tv*(k+S))
  *  x_perm     [R, H]        permuted activations (bf16; e4m3 codes for FP8)
  *  h          [R, Imax]     SwiGLU output rows (bf16; e4m3 codes for FP8)
- *  y          bf16 [R, H]   expert output rows before the weighted combine
+ *  y          fp32 [R, H]   expert output rows before the weighted combine
  *  group_offsets int32 [E+S+1]: rows of expert e are [go[e], go[e+1]); the
  *             shared expert is group E. */
 typedef struct {

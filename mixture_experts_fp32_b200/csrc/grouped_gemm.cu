@@ -8,7 +8,7 @@
 //
 //   gated (gate/up):  h[r, i] = silu(g) * u,  g = Wg[e][i,:] . x_perm[r,:],
 //                                              u = Wu[e][i,:] . x_perm[r,:]
-//   down:             y[r, o] = Wd[e][o,:] . h[r,:]
+//   down:             y[r, o] = Wd[e][o,:] . h[r,:]     (kept in fp32 for the combine)
 //
 // for every permuted row r of group e (routed experts, then the shared one).
 // Decode batches give each expert only a handful of rows, so the weights take
@@ -55,7 +55,7 @@ struct KParams {
   int rows_per_expert;
   int m_routed, m_shared;
   int up_routed, up_shared;
-  __nv_bfloat16* d;
+  void* d;          // gated: bf16 h rows; down: fp32 y rows
   int ldd;
   unsigned int* status;
   unsigned int timeout_bit;
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kAccStride;
       const int col = ti.m * BM + q * 32 + lane;
-      __nv_bfloat16* drow = p.d + (size_t)ti.row0 * p.ldd + col;
+      const size_t dofs = (size_t)ti.row0 * p.ldd + col;
       for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
         float g[16];
         tmem_ld_16(tbase + c0, g);
@@ -273,13 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c) {
             if (c0 + c < ti.nrows) {
               const float s = g[c] / (1.0f + __expf(-g[c]));
-              drow[(size_t)(c0 + c) * p.ldd] = __float2bfloat16_rn(s * u[c]);
+              static_cast<__nv_bfloat16*>(p.d)[dofs + (size_t)(c0 + c) * p.ldd] =
+                  __float2bfloat16_rn(s * u[c]);
             }
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            if (c0 + c < ti.nrows) drow[(size_t)(c0 + c) * p.ldd] = __float2bfloat16_rn(g[c]);
+            if (c0 + c < ti.nrows) static_cast<float*>(p.d)[dofs + (size_t)(c0 + c) * p.ldd] = g[c];
         }
       }
       tc_fence_before();
@@ -361,7 +362,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   p.m_shared = a.m_tiles_shared;
   p.up_routed = a.up_routed;
   p.up_shared = a.up_shared;
-  p.d = reinterpret_cast<__nv_bfloat16*>(a.d);
+  p.d = a.d;
   p.ldd = a.ldd;
   p.status = a.status;
   p.timeout_bit = a.timeout_bit;

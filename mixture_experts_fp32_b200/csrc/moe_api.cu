@@ -138,7 +138,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   p->off_rowtok = take(sizeof(int) * r_cap);
   p->off_xp = take(2 * r_cap * H);
   p->off_h = take(2 * r_cap * (size_t)imax);
-  p->off_y = take(2 * r_cap * H);
+  p->off_y = take(sizeof(float) * r_cap * H);
   p->ws_bytes = off;
   p->wait_limit_ns = 2000000000ull;
   p->device = -1;
@@ -194,7 +194,7 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
   int* rowtok = at<int>(workspace, plan->off_rowtok);
   auto* xp = at<__nv_bfloat16>(workspace, plan->off_xp);
   auto* h = at<__nv_bfloat16>(workspace, plan->off_h);
-  auto* y = at<__nv_bfloat16>(workspace, plan->off_y);
+  float* y = at<float>(workspace, plan->off_y);
   const auto* x = static_cast<const __nv_bfloat16*>(hidden);
 
   record(dbg, 0, st);

@@ -24,7 +24,7 @@ struct GroupedGemmArgs {
   const void* a_routed;
   const void* a_shared;        // may be null when there is no shared group
   const void* b;
-  void* d;                     // output rows [R_cap, ldd] bf16
+  void* d;                     // output rows [R_cap, ldd]: bf16 (gated) or fp32 (down)
   const int* group_offsets;    // [G + 1] on the device
   int E, G;                    // routed experts, total groups (E + S)
   int K_routed, K_shared, K_ld;
@@ -53,7 +53,7 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_tok
                                const int* total_rows, int R_cap, __nv_bfloat16* xp,
                                int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
-cudaError_t launch_combine(const __nv_bfloat16* y, int H, const int* inv, const float* w,
+cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
                            const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
                            cudaStream_t st);
 cudaError_t prepare_grouped_gemm_kernels();

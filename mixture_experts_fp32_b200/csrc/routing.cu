@@ -10,7 +10,7 @@
 //   bit per token) gives each pair its rank by population counts.
 // gather_rows_kernel: x_perm[r] = x[row_token[r]] with 16-byte vectors.
 // combine_kernel: out[t] = bf16( sum_j w[t,j] y[inv[t,j]] + y[inv[t,k]] ),
-//   summed in fp32 in ascending j, shared expert last; padding rows get +0.0
+//   y in fp32, summed in fp32 in ascending j, shared expert last; padding rows get +0.0
 //   (the combine phase, [SGLang] MoE 모델을 위한 Single Batch Overlap 기법,
 //   §들어가며; the fused shared expert, Step3 推論最適化 (MI308X vs H20),
 //   §最適化技術).
@@ -161,25 +161,24 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
   }
 }
 
-__device__ __forceinline__ void acc_row(float (&acc)[8], const uint4& raw, float wgt) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] = fmaf(wgt, __low2float(p[i]), acc[2 * i]);
-    acc[2 * i + 1] = fmaf(wgt, __high2float(p[i]), acc[2 * i + 1]);
-  }
+// acc[0..7] += wgt * y[8 consecutive fp32]
+__device__ __forceinline__ void acc_row(float (&acc)[8], const float* y8, float wgt) {
+  const float4 a = reinterpret_cast<const float4*>(y8)[0];
+  const float4 b = reinterpret_cast<const float4*>(y8)[1];
+  acc[0] = fmaf(wgt, a.x, acc[0]); acc[1] = fmaf(wgt, a.y, acc[1]);
+  acc[2] = fmaf(wgt, a.z, acc[2]); acc[3] = fmaf(wgt, a.w, acc[3]);
+  acc[4] = fmaf(wgt, b.x, acc[4]); acc[5] = fmaf(wgt, b.y, acc[5]);
+  acc[6] = fmaf(wgt, b.z, acc[6]); acc[7] = fmaf(wgt, b.w, acc[7]);
 }
 
-__device__ __forceinline__ void add_row(float (&acc)[8], const uint4& raw) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __low2float(p[i]);
-    acc[2 * i + 1] += __high2float(p[i]);
-  }
+__device__ __forceinline__ void add_row(float (&acc)[8], const float* y8) {
+  const float4 a = reinterpret_cast<const float4*>(y8)[0];
+  const float4 b = reinterpret_cast<const float4*>(y8)[1];
+  acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+  acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
 }
 
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ y, int H,
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, int H,
                                                       const int* __restrict__ inv,
                                                       const float* __restrict__ w,
                                                       const uint8_t* __restrict__ valid, int T,
@@ -201,12 +200,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
         for (int j = 0; j < k; ++j) {
           const int r = rows[j];
           if (r < 0) continue;
-          const uint4 raw = reinterpret_cast<const uint4*>(y + (size_t)r * H)[v];
-          acc_row(acc, raw, wts[j]);
+          acc_row(acc, y + (size_t)r * H + (size_t)v * 8, wts[j]);
         }
         if (S && rows[k] >= 0) {
-          const uint4 raw = reinterpret_cast<const uint4*>(y + (size_t)rows[k] * H)[v];
-          add_row(acc, raw);
+          add_row(acc, y + (size_t)rows[k] * H + (size_t)v * 8);
         }
       }
       uint4 o;
@@ -239,7 +236,7 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_tok
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const __nv_bfloat16* y, int H, const int* inv, const float* w,
+cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
                            const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
                            cudaStream_t st) {
   int grid = T < 148 * 16 ? T : 148 * 16;

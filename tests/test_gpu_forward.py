@@ -165,7 +165,7 @@ def test_intermediate_rows_against_fp64():
     rowtok = dev_view(v.row_token, (R,), torch.int32).numpy()
     xp = dev_view(v.x_perm, (R, w.H), torch.bfloat16)
     h = dev_view(v.h, (R, v.h_stride), torch.bfloat16)
-    y = dev_view(v.y, (R, w.H), torch.bfloat16)
+    y = dev_view(v.y, (R, w.H), torch.float32)
     assert torch.equal(xp, inp["x"][torch.from_numpy(rowtok).long()])
     x64 = inp["x"].double()
     for r in list(range(0, R, 7)) + [R - 1]:
