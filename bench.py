@@ -28,6 +28,17 @@ METRIC = "MoE-layer tokens/s; % of HBM (decode) / tensor-core (prefill) roofline
 DEFAULT_WORKLOAD = "step3_decode"
 L2_FLUSH_BYTES = 512 << 20
 
+# DRAM traffic / algorithmic bytes of one gate/up GEMM launch, from the ncu capture
+# summarised in profiles/grouped_gemm_step3_e8.md; it applies only to the kernel
+# source it was measured on (sha256 prefix), and "traffic" is null otherwise.
+GEMM_TRAFFIC = {"sha256_prefix": "44127fb7788e0211", "gate_up_ratio": 0.997}
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    p = os.path.join(ROOT, "mixture_experts_fp32_b200", "csrc", "grouped_gemm.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
 
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -44,6 +55,22 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return ws, rank, local
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Seed of a replica's own batch of hidden states (rank 0 keeps the workload's)."""
+    return seed + 1000 * rank
+
+
+def reduce_over_ranks(v: float, op: str, world: int, device) -> float:
+    """max or sum of a per-rank scalar over the process group (identity for 1 rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
 
 
 # ----------------------------------------------------------- algorithmic work
@@ -150,12 +177,13 @@ def run_native(args):
         dist.barrier()
     moe.load()
 
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     k = w.k
     # weights: drawn once (rank 0) and broadcast; activations: one batch per rank
     inp = synth.make_inputs(w, with_weights=(rank == 0))
     if ws_n > 1:
-        inp["x"] = synth.normal_bf16(w.seed + 1000 * rank, synth.STREAM_X, (w.T, w.H), w.x_sigma)
+        inp["x"] = synth.normal_bf16(replica_seed(w.seed, rank), synth.STREAM_X, (w.T, w.H),
+                                     w.x_sigma)
     d = {}
     for key in ("x", "valid", "router_w", "router_b"):
         d[key] = None if inp.get(key) is None else inp[key].to(dev)
@@ -211,11 +239,19 @@ def run_native(args):
         for e in row:
             e.record(stream)
     torch.cuda.synchronize()
+    # nvidia-smi samples every 200 ms and the timed steps take milliseconds, so the
+    # sampler also covers ~1.5 s of further (untimed) warm-up steps right before them
     clocks = ClockSampler(dev.index)
+    clocks.start()
+    t_end = time.perf_counter() + 1.5
+    while time.perf_counter() < t_end:
+        for _ in range(8):
+            flush.zero_()
+            fwd()
+        torch.cuda.synchronize()
     if ws_n > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
     t_wall = time.perf_counter()
     for i in range(K):
         flush.zero_()                      # L2 flush outside the step's events
@@ -258,25 +294,10 @@ def run_native(args):
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
 
-    def max_over_ranks(v: float) -> float:
-        if ws_n == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(v: float) -> float:
-        if ws_n == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
-
-    total_ms = max_over_ranks(total_ms)
-    e2e_total = max_over_ranks(sum(e2e_ms))
-    tokens = sum_over_ranks(float(valid_tokens))
-    gemm_ms_max = max_over_ranks(gemm_ms)
-    status = int(max_over_ranks(float(status)))
+    total_ms = reduce_over_ranks(total_ms, "max", ws_n, dev)
+    e2e_total = reduce_over_ranks(sum(e2e_ms), "max", ws_n, dev)
+    tokens = reduce_over_ranks(float(valid_tokens), "sum", ws_n, dev)
+    status = int(reduce_over_ranks(float(status), "max", ws_n, dev))
 
     peaks = measured_peaks()
     prefill = w.wtype == "fp8"
@@ -289,6 +310,9 @@ def run_native(args):
         achieved = algo["gate_up_flops"] / (gemm_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"] * (2 if w.wtype == "fp8" else 1)
         unit = "TFLOP/s"
+    traffic = None
+    if gemm_source_hash() == GEMM_TRAFFIC["sha256_prefix"] and w.wtype == "bf16":
+        traffic = GEMM_TRAFFIC["gate_up_ratio"] * algo["gate_up_bytes"]
     ms = total_ms / K
     step_roof_ms = max(algo["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
                        algo["step_flops"] / (peaks["bf16_tflops"] * 1e12)) * 1e3
@@ -308,8 +332,10 @@ def run_native(args):
                              "outside the step events; weights alone exceed L2"},
             "roofline": {"bound": bound, "kernel": "grouped_gemm gate/up + SwiGLU",
                          "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": None,
-                         "peak_source": peaks["source"]},
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes": algo["gate_up_bytes"],
+                         "algorithmic_flops": algo["gate_up_flops"],
+                         "launch_ms": gemm_ms, "peak_source": peaks["source"]},
             "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / ms,
                               "algorithmic_bytes": algo["step_bytes"],
                               "algorithmic_flops": algo["step_flops"],
@@ -371,8 +397,7 @@ def run_reference(args):
     ws_n, rank, _ = dist_env()
     if rank != 0:
         return None
-    import synth
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     rates = []
     for _ in range(max(args.warmup, 0)):
         oracle_tokens_per_s(w, min(args.cpu_seconds, 5.0))
@@ -396,6 +421,15 @@ def run_reference(args):
     return res
 
 
+def workload_of(args):
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.experts:
+        # a smaller copy of the workload (fewer experts) for profiler captures
+        w = w.with_(name=f"{w.name}_e{args.experts}", E=args.experts, k=min(w.k, args.experts))
+    return w
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,6 +439,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the number of routed experts (profiling on a smaller case)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
