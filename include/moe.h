@@ -158,6 +158,37 @@ moe_status moe_route_from_logits(moe_plan_t plan, const float *logits, const uin
                                  int T, int k, int *topk_ids, float *topk_w, int *perm,
                                  int *offsets, void *workspace, size_t ws_bytes, void *stream);
 
+/* moe_route_from_logits without a caller workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory: code running inside a framework whose memory pool owns the
+ * whole device and forbids further cudaMalloc, plain-C hosts handed only
+ * device pointers, or code that must not allocate because a CUDA graph is
+ * being captured on its stream.
+ *
+ * Results are identical to moe_route_from_logits (same kernels, same order of
+ * operations).  Its scratch (status word, group offsets, a logits copy, the
+ * inverse permutation and the row -> token map) lives in one file-scope
+ * __device__ array of MOE_STATIC_SCRATCH_BYTES that every GPU which loads the
+ * library holds until the process exits.  A call needs
+ *   256 + a(4 (E + 2)) + a(4 T E) + 2 a(4 T (k + S))  bytes,  a(n) = n rounded up to 256,
+ * and returns MOE_ERR_UNSUPPORTED, launching nothing, when that exceeds
+ * MOE_STATIC_SCRATCH_BYTES.
+ *  - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before capturing the stream into a graph.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents (each call clears what it needs cleared).  Calls whose
+ *    work overlaps on the GPU — on two streams, or from two threads — race on
+ *    it: order them on one stream.
+ *  - Its device status word is inside the array too; this routing raises no
+ *    device-side failure that moe_check_device_status would report.
+ * Arguments as in moe_route_from_logits; none of the output pointers may be NULL. */
+#define MOE_STATIC_SCRATCH_BYTES (4u << 20)
+moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float *logits,
+                                         const uint8_t *valid, int T, int k, int *topk_ids,
+                                         float *topk_w, int *perm, int *offsets, void *stream);
+
 /* Synchronises the stream, reads and clears the device status word of this
  * workspace.  *bits (may be NULL) receives the MOE_DEV_* bits that were set.
  * Returns MOE_OK if none, MOE_ERR_DEVICE otherwise. */

@@ -31,8 +31,10 @@ MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")
 
 EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
-            "moe_route_from_logits", "moe_check_device_status", "moe_get_workspace_views",
-            "moe_status_string")
+            "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
+            "moe_get_workspace_views", "moe_status_string")
+
+MOE_STATIC_SCRATCH_BYTES = 4 << 20
 
 _c_int = ctypes.c_int
 _vp = ctypes.c_void_p
@@ -90,6 +92,9 @@ def load():
     L.moe_route_from_logits.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
                                         ctypes.c_size_t, _vp]
     L.moe_route_from_logits.restype = _c_int
+    L.moe_route_from_logits_noalloc.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp,
+                                                _vp, _vp]
+    L.moe_route_from_logits_noalloc.restype = _c_int
     L.moe_check_device_status.argtypes = [_vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
     L.moe_check_device_status.restype = _c_int
     L.moe_get_workspace_views.argtypes = [_vp, _vp, ctypes.POINTER(moe_workspace_views)]
@@ -174,6 +179,16 @@ def moe_route_from_logits(plan, logits, valid, T: int, k: int, topk_ids, topk_w,
                                       _addr(topk_w), _addr(perm), _addr(offsets),
                                       _addr(workspace), ws_bytes, _stream(stream))
     _check(st, "moe_route_from_logits")
+
+
+def moe_route_from_logits_noalloc(plan, logits, valid, T: int, k: int, topk_ids, topk_w, perm,
+                                  offsets, stream=None) -> None:
+    """Routing from logits with the library's own static device scratch: for
+    callers that cannot allocate device memory (no workspace argument)."""
+    st = load().moe_route_from_logits_noalloc(plan, _addr(logits), _addr(valid), T, k,
+                                              _addr(topk_ids), _addr(topk_w), _addr(perm),
+                                              _addr(offsets), _stream(stream))
+    _check(st, "moe_route_from_logits_noalloc")
 
 
 def moe_check_device_status(plan, workspace, stream=None) -> int:

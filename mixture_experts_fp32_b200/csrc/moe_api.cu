@@ -339,3 +339,7 @@ MOE_EXPORT moe_status moe_get_workspace_views(moe_plan_t plan, void* workspace,
   v->h_stride = plan->imax;
   return MOE_OK;
 }
+
+namespace moe {
+const moe_config* plan_config(const moe_plan_s* plan) { return &plan->cfg; }
+}  // namespace moe

@@ -57,6 +57,7 @@ cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w
                            const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
                            cudaStream_t st);
 cudaError_t prepare_grouped_gemm_kernels();
+const moe_config* plan_config(const moe_plan_s* plan);
 void router_split_plan(int T, int E, int H, int num_sms, int* splits, int* kchunk);
 
 // ---------------------------------------------------------------- device side
