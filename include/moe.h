@@ -200,9 +200,13 @@ moe_status moe_check_device_status(moe_plan_t plan, void *workspace, void *strea
  *  row_token  int32 [R]     token index of each permuted row (R = Tv*(k+S))
  *  x_perm     [R, H]        permuted activations (bf16; e4m3 codes for FP8)
  *  h          [R, Imax]     SwiGLU output rows (bf16; e4m3 codes for FP8)
- *  y          fp32 [R, H]   expert output rows before the weighted combine
+ *  y          [R, H]        expert output rows before the weighted combine
+ *                           (fp32 for bf16 weights, bf16 for FP8 weights)
  *  group_offsets int32 [E+S+1]: rows of expert e are [go[e], go[e+1]); the
- *             shared expert is group E. */
+ *             shared expert is group E.
+ *  x_scale, h_scale  FP8 only (else NULL): fp32 scales of x_perm and h, one per
+ *             1x128 group, stored transposed: [H/128][C] and [Imax/128][C] with
+ *             C = T*(k+S) of the last forward. */
 typedef struct {
     int *row_token;
     void *x_perm;
@@ -210,6 +214,8 @@ typedef struct {
     void *y;
     int *group_offsets;
     int h_stride;       /* Imax = max(I, Is) elements per h row */
+    float *x_scale;
+    float *h_scale;
 } moe_workspace_views;
 moe_status moe_get_workspace_views(moe_plan_t plan, void *workspace, moe_workspace_views *views);
 

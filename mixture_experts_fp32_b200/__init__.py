@@ -59,7 +59,8 @@ class moe_debug(ctypes.Structure):
 
 class moe_workspace_views(ctypes.Structure):
     _fields_ = [("row_token", _vp), ("x_perm", _vp), ("h", _vp), ("y", _vp),
-                ("group_offsets", _vp), ("h_stride", _c_int)]
+                ("group_offsets", _vp), ("h_stride", _c_int), ("x_scale", _vp),
+                ("h_scale", _vp)]
 
 
 class MoeError(RuntimeError):

@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile ti = decode_tile(t, ts, go, p);
       const int buf = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
-      if (!mbar_wait_bounded(smem_u32(&tfull[buf]), use & 1u, p.wait_limit_ns, p.status,
+      if (!mbar_wait_bounded_warp(smem_u32(&tfull[buf]), use & 1u, p.wait_limit_ns, p.status,
                              p.timeout_bit))
         break;
       tc_fence_after();

@@ -18,7 +18,7 @@ struct moe_plan_s {
   size_t r_cap;      // max_tokens * ks_max rows
   // byte offsets inside the workspace
   size_t off_status, off_goff, off_partial, off_logits, off_ids, off_w, off_perm, off_inv,
-      off_rowtok, off_xp, off_h, off_y;
+      off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
   unsigned long long wait_limit_ns;
   int device;
   int num_sms;
@@ -50,7 +50,9 @@ moe_status ensure_device(moe_plan_s* p) {
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
   if (dev < 64 && !((prepared_mask >> dev) & 1ull)) {
-    if (moe::prepare_grouped_gemm_kernels() != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::prepare_grouped_gemm_kernels() != cudaSuccess ||
+        moe::prepare_grouped_gemm_fp8_kernels() != cudaSuccess)
+      return MOE_ERR_CUDA;
     prepared_mask |= 1ull << dev;
   }
   p->num_sms = sms;
@@ -107,7 +109,6 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   if (c.hidden % 128 != 0 || c.inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c.num_shared == 1 && c.shared_inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c.hidden > 65536 || c.inter > 65536 || c.shared_inter > 65536) return MOE_ERR_UNSUPPORTED;
-  if (c.wtype != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;   // e4m3 block-scale path not built yet
   const int S = c.num_shared;
   const int imax = S && c.shared_inter > c.inter ? c.shared_inter : c.inter;
   const size_t T = (size_t)c.max_tokens, E = (size_t)c.num_experts, H = (size_t)c.hidden;
@@ -136,9 +137,21 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   p->off_perm = take(sizeof(int) * T * c.top_k_max);
   p->off_inv = take(sizeof(int) * T * ks);
   p->off_rowtok = take(sizeof(int) * r_cap);
-  p->off_xp = take(2 * r_cap * H);
-  p->off_h = take(2 * r_cap * (size_t)imax);
-  p->off_y = take(sizeof(float) * r_cap * H);
+  if (c.wtype == MOE_W_BF16) {
+    // bf16 permuted rows and h; fp32 expert outputs
+    p->off_xp = take(2 * r_cap * H);
+    p->off_sx = 0;
+    p->off_h = take(2 * r_cap * (size_t)imax);
+    p->off_sh = 0;
+    p->off_y = take(sizeof(float) * r_cap * H);
+  } else {
+    // e4m3 permuted rows and h with transposed 1x128 scales; bf16 expert outputs
+    p->off_xp = take(r_cap * H);
+    p->off_sx = take(sizeof(float) * (H / 128) * r_cap);
+    p->off_h = take(r_cap * (size_t)imax);
+    p->off_sh = take(sizeof(float) * ((size_t)imax / 128) * r_cap);
+    p->off_y = take(2 * r_cap * H);
+  }
   p->ws_bytes = off;
   p->wait_limit_ns = 2000000000ull;
   p->device = -1;
@@ -174,6 +187,10 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
       (S && (!aligned16(wts->ws_gate_up) || !aligned16(wts->ws_down))))
     return MOE_ERR_INVALID_ARG;
   if ((wts->router_b != nullptr && (reinterpret_cast<uintptr_t>(wts->router_b) & 3u)) != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c.wtype == MOE_W_FP8_E4M3_B128 &&
+      (wts->s_gate_up == nullptr || wts->s_down == nullptr ||
+       (S && (wts->ss_gate_up == nullptr || wts->ss_down == nullptr))))
     return MOE_ERR_INVALID_ARG;
   s = ensure_device(plan);
   if (s != MOE_OK) return s;
@@ -212,59 +229,129 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
   s = check_launch(moe::launch_route(ids, valid, T, E, k, S, goff, perm, inv, rowtok, status, st));
   if (s != MOE_OK) return s;
   record(dbg, 3, st);
-  s = check_launch(moe::launch_gather_rows(x, H, rowtok, goff + G, R_cap, xp, plan->num_sms, st));
+  const bool fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
+  if (!fp8) {
+    s = check_launch(
+        moe::launch_gather_rows(x, H, rowtok, goff + G, R_cap, xp, plan->num_sms, st));
+  } else {
+    s = check_launch(moe::launch_quant_gather(x, H, rowtok, goff + G, R_cap,
+                                              at<uint8_t>(workspace, plan->off_xp),
+                                              at<float>(workspace, plan->off_sx), plan->num_sms,
+                                              st));
+  }
   if (s != MOE_OK) return s;
   record(dbg, 4, st);
 
-  moe::GroupedGemmArgs ga;
-  memset(&ga, 0, sizeof(ga));
-  ga.a_routed = wts->w_gate_up;
-  ga.a_shared = S ? wts->ws_gate_up : nullptr;
-  ga.b = xp;
-  ga.d = h;
-  ga.group_offsets = goff;
-  ga.E = E;
-  ga.G = G;
-  ga.K_routed = H;
-  ga.K_shared = H;
-  ga.K_ld = H;
-  ga.rows_per_expert = 2 * I;
-  ga.m_tiles_routed = I / 128;
-  ga.m_tiles_shared = S ? Is / 128 : 0;
-  ga.up_routed = I;
-  ga.up_shared = Is;
-  ga.ldd = plan->imax;
-  ga.R_cap = R_cap;
-  ga.gated = true;
-  ga.status = status;
-  ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_GATE_UP;
-  ga.wait_limit_ns = plan->wait_limit_ns;
-  ga.num_ctas = plan->num_sms;
-  s = check_launch(moe::launch_grouped_gemm(ga, st));
-  if (s != MOE_OK) return s;
-  record(dbg, 5, st);
+  if (!fp8) {
+    moe::GroupedGemmArgs ga;
+    memset(&ga, 0, sizeof(ga));
+    ga.a_routed = wts->w_gate_up;
+    ga.a_shared = S ? wts->ws_gate_up : nullptr;
+    ga.b = xp;
+    ga.d = h;
+    ga.group_offsets = goff;
+    ga.E = E;
+    ga.G = G;
+    ga.K_routed = H;
+    ga.K_shared = H;
+    ga.K_ld = H;
+    ga.rows_per_expert = 2 * I;
+    ga.m_tiles_routed = I / 128;
+    ga.m_tiles_shared = S ? Is / 128 : 0;
+    ga.up_routed = I;
+    ga.up_shared = Is;
+    ga.ldd = plan->imax;
+    ga.R_cap = R_cap;
+    ga.gated = true;
+    ga.status = status;
+    ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_GATE_UP;
+    ga.wait_limit_ns = plan->wait_limit_ns;
+    ga.num_ctas = plan->num_sms;
+    s = check_launch(moe::launch_grouped_gemm(ga, st));
+    if (s != MOE_OK) return s;
+    record(dbg, 5, st);
 
-  ga.a_routed = wts->w_down;
-  ga.a_shared = S ? wts->ws_down : nullptr;
-  ga.b = h;
-  ga.d = y;
-  ga.K_routed = I;
-  ga.K_shared = S ? Is : 0;
-  ga.K_ld = plan->imax;
-  ga.rows_per_expert = H;
-  ga.m_tiles_routed = H / 128;
-  ga.m_tiles_shared = S ? H / 128 : 0;
-  ga.up_routed = 0;
-  ga.up_shared = 0;
-  ga.ldd = H;
-  ga.gated = false;
-  ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
-  s = check_launch(moe::launch_grouped_gemm(ga, st));
-  if (s != MOE_OK) return s;
-  record(dbg, 6, st);
+    ga.a_routed = wts->w_down;
+    ga.a_shared = S ? wts->ws_down : nullptr;
+    ga.b = h;
+    ga.d = y;
+    ga.K_routed = I;
+    ga.K_shared = S ? Is : 0;
+    ga.K_ld = plan->imax;
+    ga.rows_per_expert = H;
+    ga.m_tiles_routed = H / 128;
+    ga.m_tiles_shared = S ? H / 128 : 0;
+    ga.up_routed = 0;
+    ga.up_shared = 0;
+    ga.ldd = H;
+    ga.gated = false;
+    ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
+    s = check_launch(moe::launch_grouped_gemm(ga, st));
+    if (s != MOE_OK) return s;
+    record(dbg, 6, st);
 
-  s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S,
-                                       static_cast<__nv_bfloat16*>(out), st));
+    s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S,
+                                         static_cast<__nv_bfloat16*>(out), st));
+  } else {
+    moe::GroupedGemmFp8Args fa;
+    memset(&fa, 0, sizeof(fa));
+    fa.a_routed = wts->w_gate_up;
+    fa.a_shared = S ? wts->ws_gate_up : nullptr;
+    fa.sa_routed = wts->s_gate_up;
+    fa.sa_shared = S ? wts->ss_gate_up : nullptr;
+    fa.b = at<uint8_t>(workspace, plan->off_xp);
+    fa.sb = at<float>(workspace, plan->off_sx);
+    fa.d = at<uint8_t>(workspace, plan->off_h);
+    fa.sd = at<float>(workspace, plan->off_sh);
+    fa.group_offsets = goff;
+    fa.E = E;
+    fa.G = G;
+    fa.K_routed = H;
+    fa.K_shared = H;
+    fa.K_ld = H;
+    fa.rows_per_expert = 2 * I;
+    fa.m_tiles_routed = I / 128;
+    fa.m_tiles_shared = S ? Is / 128 : 0;
+    fa.up_routed = I;
+    fa.up_shared = Is;
+    fa.ldd = plan->imax;
+    fa.R_cap = R_cap;
+    fa.gated = true;
+    fa.status = status;
+    fa.timeout_bit = MOE_DEV_WAIT_TIMEOUT_GATE_UP;
+    fa.wait_limit_ns = plan->wait_limit_ns;
+    fa.num_ctas = plan->num_sms;
+    s = check_launch(moe::launch_grouped_gemm_fp8(fa, st));
+    if (s != MOE_OK) return s;
+    record(dbg, 5, st);
+
+    auto* y16 = at<__nv_bfloat16>(workspace, plan->off_y);
+    fa.a_routed = wts->w_down;
+    fa.a_shared = S ? wts->ws_down : nullptr;
+    fa.sa_routed = wts->s_down;
+    fa.sa_shared = S ? wts->ss_down : nullptr;
+    fa.b = at<uint8_t>(workspace, plan->off_h);
+    fa.sb = at<float>(workspace, plan->off_sh);
+    fa.d = y16;
+    fa.sd = nullptr;
+    fa.K_routed = I;
+    fa.K_shared = S ? Is : 0;
+    fa.K_ld = plan->imax;
+    fa.rows_per_expert = H;
+    fa.m_tiles_routed = H / 128;
+    fa.m_tiles_shared = S ? H / 128 : 0;
+    fa.up_routed = 0;
+    fa.up_shared = 0;
+    fa.ldd = H;
+    fa.gated = false;
+    fa.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
+    s = check_launch(moe::launch_grouped_gemm_fp8(fa, st));
+    if (s != MOE_OK) return s;
+    record(dbg, 6, st);
+
+    s = check_launch(moe::launch_combine_bf16y(y16, H, inv, w, valid, T, k, S,
+                                               static_cast<__nv_bfloat16*>(out), st));
+  }
   if (s != MOE_OK) return s;
   record(dbg, 7, st);
 
@@ -337,6 +424,9 @@ MOE_EXPORT moe_status moe_get_workspace_views(moe_plan_t plan, void* workspace,
   v->y = at<void>(workspace, plan->off_y);
   v->group_offsets = at<int>(workspace, plan->off_goff);
   v->h_stride = plan->imax;
+  const bool fp8 = plan->cfg.wtype == MOE_W_FP8_E4M3_B128;
+  v->x_scale = fp8 ? at<float>(workspace, plan->off_sx) : nullptr;
+  v->h_scale = fp8 ? at<float>(workspace, plan->off_sh) : nullptr;
   return MOE_OK;
 }
 

@@ -40,6 +40,41 @@ struct GroupedGemmArgs {
   int num_ctas;
 };
 
+// e4m3 grouped GEMM with one fp32 scale per 128x128 weight block and per 1x128
+// activation group (K blocks of 128).
+struct GroupedGemmFp8Args {
+  const void* a_routed;        // e4m3 [E * rows_per_expert, K_routed]
+  const void* a_shared;        // e4m3 [rows_shared, K_shared] or null
+  const float* sa_routed;      // [E, rows_per_expert / 128, K_routed / 128]
+  const float* sa_shared;      // [rows_shared / 128, K_shared / 128]
+  const void* b;               // e4m3 activation rows [R_cap, K_ld]
+  const float* sb;             // their scales, transposed [K_ld / 128, R_cap]
+  void* d;                     // gated: e4m3 h [R_cap, ldd]; down: bf16 y [R_cap, ldd]
+  float* sd;                   // gated: h scales, transposed [ldd / 128, R_cap]
+  const int* group_offsets;
+  int E, G;
+  int K_routed, K_shared, K_ld;
+  int rows_per_expert;
+  int m_tiles_routed, m_tiles_shared;
+  int up_routed, up_shared;
+  int ldd;
+  int R_cap;
+  bool gated;
+  unsigned int* status;
+  unsigned int timeout_bit;
+  unsigned long long wait_limit_ns;
+  int num_ctas;
+};
+
+cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
+                                const int* total_rows, int R_cap, uint8_t* xq, float* sxT,
+                                int num_sms, cudaStream_t st);
+cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st);
+cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
+                                 const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                                 cudaStream_t st);
+cudaError_t prepare_grouped_gemm_fp8_kernels();
+
 cudaError_t launch_router_logits(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
                                  const float* Wr, int E, float* partial, int splits, int kchunk,
                                  cudaStream_t st);
@@ -122,6 +157,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// The same wait taken by a whole warp: every lane polls, the warp agrees by
+// vote, so a warp never splits between "done" and "expired".
+__device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t parity,
+                                                       unsigned long long limit_ns,
+                                                       unsigned int* status, unsigned int bit) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__any_sync(0xffffffffu, global_timer_ns() - t0 >= limit_ns)) {
+      if ((threadIdx.x & 31) == 0) atomicOr(status, bit);
+      return false;
+    }
+  }
+}
+
 // L2 eviction-priority policies for TMA loads.
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -180,6 +231,26 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (e4m3 inputs, fp32 accumulate), K = 32.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, e4m3 A and B (format 0),
+// both K-major, M = 128, N = n (multiple of 16, 16..256).
+__device__ __forceinline__ uint32_t idesc_e4m3_m128(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Arrive on an mbarrier once every tcgen05 operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -201,6 +272,19 @@ __device__ __forceinline__ void tmem_ld_16(uint32_t taddr, float (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Each thread of the warp reads 8 consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_ld_8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA

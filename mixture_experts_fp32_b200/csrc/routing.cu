@@ -14,6 +14,8 @@
 //   (the combine phase, [SGLang] MoE 모델을 위한 Single Batch Overlap 기법,
 //   §들어가며; the fused shared expert, Step3 推論最適化 (MI308X vs H20),
 //   §最適化技術).
+#include <cuda_fp8.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -161,24 +163,24 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
   }
 }
 
-// acc[0..7] += wgt * y[8 consecutive fp32]
-__device__ __forceinline__ void acc_row(float (&acc)[8], const float* y8, float wgt) {
+// Eight consecutive expert outputs as fp32 (fp32 rows, or bf16 rows of the FP8 path).
+__device__ __forceinline__ void load8(const float* y8, float (&v)[8]) {
   const float4 a = reinterpret_cast<const float4*>(y8)[0];
   const float4 b = reinterpret_cast<const float4*>(y8)[1];
-  acc[0] = fmaf(wgt, a.x, acc[0]); acc[1] = fmaf(wgt, a.y, acc[1]);
-  acc[2] = fmaf(wgt, a.z, acc[2]); acc[3] = fmaf(wgt, a.w, acc[3]);
-  acc[4] = fmaf(wgt, b.x, acc[4]); acc[5] = fmaf(wgt, b.y, acc[5]);
-  acc[6] = fmaf(wgt, b.z, acc[6]); acc[7] = fmaf(wgt, b.w, acc[7]);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* y8, float (&v)[8]) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(y8);
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __low2float(p[i]);
+    v[2 * i + 1] = __high2float(p[i]);
+  }
 }
 
-__device__ __forceinline__ void add_row(float (&acc)[8], const float* y8) {
-  const float4 a = reinterpret_cast<const float4*>(y8)[0];
-  const float4 b = reinterpret_cast<const float4*>(y8)[1];
-  acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-  acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
-}
-
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, int H,
+template <typename YT>
+__global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, int H,
                                                       const int* __restrict__ inv,
                                                       const float* __restrict__ w,
                                                       const uint8_t* __restrict__ valid, int T,
@@ -200,10 +202,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         for (int j = 0; j < k; ++j) {
           const int r = rows[j];
           if (r < 0) continue;
-          acc_row(acc, y + (size_t)r * H + (size_t)v * 8, wts[j]);
+          float yv[8];
+          load8(y + (size_t)r * H + (size_t)v * 8, yv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(wts[j], yv[i], acc[i]);
         }
         if (S && rows[k] >= 0) {
-          add_row(acc, y + (size_t)rows[k] * H + (size_t)v * 8);
+          float yv[8];
+          load8(y + (size_t)rows[k] * H + (size_t)v * 8, yv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += yv[i];
         }
       }
       uint4 o;
@@ -213,6 +221,42 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       dst[v] = o;
     }
     __syncthreads();
+  }
+}
+
+// FP8 path: x_perm[r] = e4m3 codes of x[row_token[r]] with one scale per 1x128
+// group: s = amax / 448 (1 when amax = 0), q = e4m3_rne_sat(x / s), both fp32
+// divisions correctly rounded.  Scales are stored transposed, sxT[g][r], so
+// that a K block's scales for consecutive rows are contiguous.
+__global__ void __launch_bounds__(256) quant_gather_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           int H,
+                                                           const int* __restrict__ row_token,
+                                                           const int* __restrict__ total_rows,
+                                                           int R_cap, uint8_t* __restrict__ xq,
+                                                           float* __restrict__ sxT) {
+  const int R = *total_rows;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int groups = H / 128;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    const int t = row_token[r];
+    for (int g = warp; g < groups; g += blockDim.x / 32) {
+      const uint2 raw =
+          *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)g * 128 + lane * 4);
+      const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+      const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+      const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
+      float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
+                  << (8 * i);
+      *reinterpret_cast<uint32_t*>(xq + (size_t)r * H + (size_t)g * 128 + lane * 4) = packed;
+      if (lane == 0) sxT[(size_t)g * R_cap + r] = s;
+    }
   }
 }
 
@@ -241,7 +285,26 @@ cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w
                            cudaStream_t st) {
   int grid = T < 148 * 16 ? T : 148 * 16;
   if (grid < 1) grid = 1;
-  combine_kernel<<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  combine_kernel<float><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
+                                 const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                                 cudaStream_t st) {
+  int grid = T < 148 * 16 ? T : 148 * 16;
+  if (grid < 1) grid = 1;
+  combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
+                                const int* total_rows, int R_cap, uint8_t* xq, float* sxT,
+                                int num_sms, cudaStream_t st) {
+  int grid = num_sms * 8;
+  if (grid > R_cap) grid = R_cap;
+  if (grid < 1) grid = 1;
+  quant_gather_kernel<<<grid, 256, 0, st>>>(x, H, row_token, total_rows, R_cap, xq, sxT);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@ from moe_harness import check_against_oracle, plan_for, run_forward, to_device
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["step3_decode", "deepseek_decode", "dp_padded"]
+FULL = ["step3_decode", "deepseek_decode", "dp_padded", "fp8_prefill"]
 
 
 def sample_rows(valid: np.ndarray, n_random: int = 6, seed: int = 0) -> np.ndarray:
