@@ -314,8 +314,13 @@ def run_native(args):
     if gemm_source_hash() == GEMM_TRAFFIC["sha256_prefix"] and w.wtype == "bf16":
         traffic = GEMM_TRAFFIC["gate_up_ratio"] * algo["gate_up_bytes"]
     ms = total_ms / K
+    # expert flops at the weights' dtype peak (FP8: twice the measured bf16 figure,
+    # the nominal dense ratio), router flops (fp32 logits) at the bf16 figure
+    mm_peak = peaks["bf16_tflops"] * (2 if w.wtype == "fp8" else 1) * 1e12
     step_roof_ms = max(algo["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
-                       algo["step_flops"] / (peaks["bf16_tflops"] * 1e12)) * 1e3
+                       algo["expert_flops"] / mm_peak
+                       + (algo["step_flops"] - algo["expert_flops"]) / (peaks["bf16_tflops"] * 1e12)
+                       ) * 1e3
 
     result = None
     if rank == 0:

@@ -205,8 +205,7 @@ moe_status moe_check_device_status(moe_plan_t plan, void *workspace, void *strea
  *  group_offsets int32 [E+S+1]: rows of expert e are [go[e], go[e+1]); the
  *             shared expert is group E.
  *  x_scale, h_scale  FP8 only (else NULL): fp32 scales of x_perm and h, one per
- *             1x128 group, stored transposed: [H/128][C] and [Imax/128][C] with
- *             C = T*(k+S) of the last forward. */
+ *             1x128 group, row-major: [R][H/128] and [R][Imax/128]. */
 typedef struct {
     int *row_token;
     void *x_perm;
@@ -220,6 +219,10 @@ typedef struct {
 moe_status moe_get_workspace_views(moe_plan_t plan, void *workspace, moe_workspace_views *views);
 
 const char *moe_status_string(moe_status s);
+
+/* Text of the last CUDA runtime error behind an MOE_ERR_CUDA returned to this
+ * thread ("no error" if none). */
+const char *moe_last_cuda_error_string(void);
 
 #ifdef __cplusplus
 }

@@ -32,7 +32,7 @@ STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm
 
 EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
             "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
-            "moe_get_workspace_views", "moe_status_string")
+            "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string")
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
 
@@ -66,7 +66,8 @@ class moe_workspace_views(ctypes.Structure):
 class MoeError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {moe_status_string(status)} ({status})")
+        detail = f": {moe_last_cuda_error_string()}" if status == MOE_ERR_CUDA else ""
+        super().__init__(f"{where}: {moe_status_string(status)} ({status}){detail}")
 
 
 _lib = None
@@ -102,6 +103,8 @@ def load():
     L.moe_get_workspace_views.restype = _c_int
     L.moe_status_string.argtypes = [_c_int]
     L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_last_cuda_error_string.argtypes = []
+    L.moe_last_cuda_error_string.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -131,6 +134,10 @@ def _check(status: int, where: str):
 
 def moe_status_string(status: int) -> str:
     return load().moe_status_string(status).decode()
+
+
+def moe_last_cuda_error_string() -> str:
+    return load().moe_last_cuda_error_string().decode()
 
 
 def moe_plan_create(cfg: moe_config):

@@ -5,26 +5,34 @@
 // ATOM, kernels fusionnés et montée en charge, introduction): weights carry one
 // fp32 scale per 128x128 block, activations one per 1x128 group, so
 //
-//   acc[m, n] = sum_kb  s_w[m/128, kb] * s_a[n, kb] * sum_{k in kb} qw[m, k] * qa[n, k].
+//   acc[t, n] = sum_kb  s_a[t, kb] * s_w[n/128, kb] * sum_{k in kb} qa[t, k] * qw[n, k].
 //
 // The scale changes every 128 K, and arbitrary fp32 scales cannot be given to
 // the tensor core's block-scaled kinds (they take power-of-two scales), so each
 // 128-wide K block is multiplied (kind::f8f6f4, exact products, fp32 sums) into
 // a fresh tensor-memory partial, and the epilogue warps fold every partial into
-// fp32 register accumulators with its scale product ("promotion").  Two partial
+// fp32 register accumulators with its scale ("promotion").  Two partial
 // buffers let the tensor core run one K block ahead of the promotion.
 //
-//   gated: a tile owns 128 gate rows and the matching 128 up rows of one expert
-//          (one 128-row scale block each) and up to 128 rows of activations;
-//          after the last K block h = silu(g) * u is quantised per 1x128 group
-//          (the tile's 128 columns of h are exactly one group) into e4m3 codes
-//          with an fp32 scale, ready for the down GEMM.
-//   down:  a tile owns 128 output features (one scale block) and up to 256
-//          rows; y is written in bf16.
+// Rows of activations take the MMA's M side (128 per tile) and weight rows its
+// N side (256): a TMEM lane is one activation row, so the activation scale of a
+// K block is one register per thread and the weight scale one per 128 columns;
+// promotion is one FMA per value, and each thread writes its row contiguously.
 //
-// Warp roles (576 threads): warp 0 issues TMA loads, warp 1 owns tensor memory
-// and issues the MMAs, warps 2-17 promote and finish (warp w reads TMEM lanes
-// 32*(w%4)... and one quarter of the tile's columns).  Waits are bounded.
+//   gated: a tile owns 128 features of h for up to 128 rows of one group: the
+//          B operand stacks the matching 128 gate rows and 128 up rows (N = 256),
+//          so g and u of a feature sit in the same TMEM lane.  After the last K
+//          block h = silu(g) * u is quantised per 1x128 group (the tile's 128
+//          features are one group) into e4m3 codes and an fp32 scale.
+//   down:  a tile owns up to 256 output features (two weight scale blocks) for
+//          up to 128 rows; y is written in bf16.
+//
+// Three warpgroups (384 threads).  Warpgroup 0: warp 0 issues TMA loads, warp 1
+// owns tensor memory and issues the MMAs; it gives registers back
+// (setmaxnreg.dec).  Warpgroups 1 and 2 (8 warps) promote and finish, with the
+// registers warpgroup 0 released: warp w reads TMEM lanes 32*(w%4)... and one
+// half of the tile's columns, 128 fp32 accumulators a thread.  Every wait is
+// bounded and suspends rather than spins.
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
@@ -33,50 +41,55 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 128;           // e4m3 elements (= bytes) per K block: one scale group
-constexpr int kEpiWarps = 16;
-constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr int BMT = 128;           // activation rows per tile (MMA M)
+constexpr int BK = 128;            // e4m3 elements (= bytes) per K block: one scale group
+constexpr int BNW = 256;           // weight rows per tile (MMA N)
+constexpr int kEpiWarps = 8;       // two per TMEM lane quadrant, each half of the columns
+constexpr int kThreads = 384;
+// 12 warps leave each SM sub-partition three warps: 168 registers a thread at
+// launch.  Warpgroup 0 drops to 56, warpgroups 1-2 rise to 224:
+// 128 * 56 + 256 * 224 = 384 * 168 = 64512 registers, and per sub-partition
+// 56 + 224 + 224 = 504 <= 512.
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 56;
+constexpr int kEpilogueRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kEpilogueRegs == kThreads * kLaunchRegs,
+              "register shares must add up to the launch's registers");
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPartStride = 256;  // TMEM columns between the two partial buffers
+constexpr int kPartStride = 256;   // TMEM columns between the two partial buffers
+constexpr int A_BYTES = BMT * BK;  // 16 KB
+constexpr int B_BYTES = BNW * BK;  // 32 KB
+constexpr int STAGES = 4;
+constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
+constexpr int RED_BYTES = 2 * BMT * 2 * 4;    // h amax halves [tile parity][row][half]
+constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 2048;
 constexpr unsigned long long kTeardownLimitNs = 1000000000ull;
-
-template <bool GATED>
-struct Cfg8 {
-  static constexpr int BN = 128;                          // activation rows per tile
-  static constexpr int COLS = BN / 4;                     // columns per epilogue warp
-  static constexpr int A_BYTES = (GATED ? 2 : 1) * BM * BK;
-  static constexpr int B_BYTES = BN * BK;
-  static constexpr int STAGES = 4;
-  static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
-  static constexpr int RED_BYTES = GATED ? 2 * 4 * BN * 4 : 0;   // column maxima [2][4][BN]
-  static constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 2048;
-};
 
 struct KParams8 {
   const int* group_offsets;
   int E, G;
   int kb_routed, kb_shared;
-  int rows_per_expert;
-  int m_routed, m_shared;
-  int up_routed, up_shared;
-  const float* sa_routed;
-  const float* sa_shared;
-  const float* sb;
-  void* d;
-  float* sd;
+  int rows_per_expert;            // weight rows of one routed expert
+  int ft_routed, ft_shared;       // feature tiles per group
+  int feat_routed, feat_shared;   // features per group (down: H; gated: I or Is)
+  int up_routed, up_shared;       // gated: row offset of the up half
+  const float* sw_routed;         // [E, rows_per_expert/128, kb_routed]
+  const float* sw_shared;         // [rows_shared/128, kb_shared]
+  const float* sa;                // activation scales [R_cap, sa_ld] (row-major)
+  int sa_ld;
+  void* d;                        // gated: e4m3 h [R_cap, ldd]; down: bf16 y [R_cap, ldd]
+  float* sd;                      // gated: h scales [R_cap, ldd/128]
   int ldd;
-  int R_cap;
   unsigned int* status;
   unsigned int timeout_bit;
   unsigned long long wait_limit_ns;
 };
 
 struct Tile8 {
-  int g, m, row0, nrows, n_mma, k_blocks;
+  int g, f0, nfeat, row0, nrows, k_blocks, row_tiles;
 };
 
-template <int BN>
+template <bool GATED>
 __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* go,
                                               const KParams8& p) {
   int lo = 0, hi = p.G;
@@ -86,39 +99,45 @@ __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* g
   }
   Tile8 ti;
   ti.g = lo;
+  const bool routed = lo < p.E;
   const int gbeg = go[lo], gend = go[lo + 1];
-  const int nt = (gend - gbeg + BN - 1) / BN;
+  const int rt = (gend - gbeg + BMT - 1) / BMT;
   const int local = t - ts[lo];
-  ti.m = local / nt;
-  const int n = local - ti.m * nt;
-  ti.row0 = gbeg + n * BN;
-  ti.nrows = min(BN, gend - ti.row0);
-  ti.n_mma = (ti.nrows + 15) & ~15;
-  ti.k_blocks = lo < p.E ? p.kb_routed : p.kb_shared;
+  const int f = local / rt;                    // feature tile outer, row tile inner
+  const int r = local - f * rt;
+  const int fpt = GATED ? 128 : BNW;           // features per tile
+  const int feats = routed ? p.feat_routed : p.feat_shared;
+  ti.f0 = f * fpt;
+  ti.nfeat = min(fpt, feats - ti.f0);
+  ti.row0 = gbeg + r * BMT;
+  ti.nrows = min(BMT, gend - ti.row0);
+  ti.k_blocks = routed ? p.kb_routed : p.kb_shared;
+  ti.row_tiles = rt;
   return ti;
 }
 
-__device__ __forceinline__ uint8_t e4m3_of(float v) {
-  return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
 }
 
 template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,
-                            const __grid_constant__ CUtensorMap tmAs,
-                            const __grid_constant__ CUtensorMap tmB, const KParams8 p) {
-  using C = Cfg8<GATED>;
-  constexpr int BN = C::BN;
+    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA,    // activation rows
+                            const __grid_constant__ CUtensorMap tmW,    // routed weights
+                            const __grid_constant__ CUtensorMap tmWs,   // shared weights
+                            const KParams8 p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* a_smem = base;
-  uint8_t* b_smem = base + C::STAGES * C::A_BYTES;
-  float* red = reinterpret_cast<float*>(base + C::DATA_BYTES);   // [tile parity][quadrant][column]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::DATA_BYTES + C::RED_BYTES);
+  uint8_t* b_smem = base + STAGES * A_BYTES;
+  float* red = reinterpret_cast<float*>(base + DATA_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + DATA_BYTES + RED_BYTES);
   uint64_t* full = bars;
-  uint64_t* empty = bars + C::STAGES;
-  uint64_t* pfull = bars + 2 * C::STAGES;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* pfull = bars + 2 * STAGES;
   uint64_t* pempty = pfull + 2;
   uint64_t* teardown = pempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
@@ -128,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int* go = p.group_offsets;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
@@ -139,21 +158,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(teardown), 1);
     fence_mbarrier_init();
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmAs);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmWs);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
   if (warp == 2) {
+    // tile prefix over groups: ceil(rows / 128) row tiles x feature tiles
     int running = 0;
     for (int b0 = 0; b0 < p.G; b0 += 32) {
       const int g = b0 + lane;
       int cnt = 0;
       if (g < p.G) {
         const int rows = go[g + 1] - go[g];
-        cnt = (g < p.E ? p.m_routed : p.m_shared) * ((rows + BN - 1) / BN);
+        cnt = (g < p.E ? p.ft_routed : p.ft_shared) * ((rows + BMT - 1) / BMT);
       }
       int incl = cnt;
 #pragma unroll
@@ -172,144 +192,170 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int total = ts[p.G];
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_a = policy_evict_first();
-      const uint64_t pol_b = policy_evict_last();
+  if (warp < 4) {
+    regs_dec<kProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      // A group with one row tile reads its weights once (evict first) and its
+      // rows once per feature tile (evict last); larger groups reuse both from
+      // L2 across neighbouring tiles (evict normal).
+      const uint64_t pol_first = policy_evict_first();
+      const uint64_t pol_last = policy_evict_last();
+      const uint64_t pol_normal = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile8 ti = decode_tile8<BN>(t, ts, go, p);
+        const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
         const bool routed = ti.g < p.E;
-        const CUtensorMap* am = routed ? &tmA : &tmAs;
-        const int arow = (routed ? ti.g * p.rows_per_expert : 0) + ti.m * BM;
+        const CUtensorMap* wm = routed ? &tmW : &tmWs;
+        const int wrow = (routed ? ti.g * p.rows_per_expert : 0) + ti.f0;
         const int up = routed ? p.up_routed : p.up_shared;
-        const uint32_t bytes = C::A_BYTES + ti.n_mma * BK;
+        const int nb = GATED ? 2 : (ti.nfeat + 127) / 128;      // 128-row weight boxes
+        const uint32_t bytes = A_BYTES + nb * 128 * BK;
+        const uint64_t pol_a = ti.row_tiles == 1 ? pol_last : pol_normal;
+        const uint64_t pol_w = ti.row_tiles == 1 ? pol_first : pol_normal;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
-          if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, p.wait_limit_ns, p.status,
-                                 p.timeout_bit)) {
+          if (!mbar_wait_sleep(smem_u32(&empty[stage]), phase ^ 1u, p.wait_limit_ns, p.status,
+                               p.timeout_bit)) {
             ok = false;
             break;
           }
           const uint32_t fb = smem_u32(&full[stage]);
           mbar_arrive_expect_tx(fb, bytes);
-          const uint32_t a_dst = smem_u32(a_smem + stage * C::A_BYTES);
-          tma_load_2d(a_dst, am, kb * BK, arow, fb, pol_a);
-          if (GATED) tma_load_2d(a_dst + BM * BK, am, kb * BK, arow + up, fb, pol_a);
-          const uint32_t b_dst = smem_u32(b_smem + stage * C::B_BYTES);
-          for (int nb = 0; nb < ti.n_mma / 16; ++nb)
-            tma_load_2d(b_dst + nb * 16 * BK, &tmB, kb * BK, ti.row0 + nb * 16, fb, pol_b);
+          tma_load_2d(smem_u32(a_smem + stage * A_BYTES), &tmA, kb * BK, ti.row0, fb, pol_a);
+          const uint32_t b_dst = smem_u32(b_smem + stage * B_BYTES);
+          if (GATED) {
+            tma_load_2d(b_dst, wm, kb * BK, wrow, fb, pol_w);
+            tma_load_2d(b_dst + 128 * BK, wm, kb * BK, wrow + up, fb, pol_w);
+          } else {
+            for (int j = 0; j < nb; ++j)
+              tma_load_2d(b_dst + j * 128 * BK, wm, kb * BK, wrow + 128 * j, fb, pol_w);
+          }
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      for (int s = 0; s < C::STAGES; ++s)
+      for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1u)
-          mbar_wait_bounded(smem_u32(&full[s]), (parity >> s) & 1u, kTeardownLimitNs, p.status,
-                            p.timeout_bit);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+          mbar_wait_sleep(smem_u32(&full[s]), (parity >> s) & 1u, kTeardownLimitNs, p.status,
+                          p.timeout_bit);
+    } else if (warp == 1 && lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       uint32_t kcount = 0;          // K blocks issued so far: partial buffer = kcount & 1
       bool ok = true, any = false;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile8 ti = decode_tile8<BN>(t, ts, go, p);
-        const uint32_t idesc = idesc_e4m3_m128(ti.n_mma);
+        const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
+        const int n = GATED ? 256 : ((ti.nfeat + 127) / 128) * 128;
+        const uint32_t idesc = idesc_e4m3_m128(n);
         for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
           const uint32_t pb = kcount & 1u;
           const uint32_t use = kcount >> 1;
-          if (!mbar_wait_bounded(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns,
-                                 p.status, p.timeout_bit) ||
-              !mbar_wait_bounded(smem_u32(&full[stage]), phase, p.wait_limit_ns, p.status,
-                                 p.timeout_bit)) {
+          if (!mbar_wait_sleep(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns, p.status,
+                               p.timeout_bit) ||
+              !mbar_wait_sleep(smem_u32(&full[stage]), phase, p.wait_limit_ns, p.status,
+                               p.timeout_bit)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t d0 = tmem_base + pb * kPartStride;
-          const uint64_t a_desc = smem_desc_sw128(smem_u32(a_smem + stage * C::A_BYTES));
-          const uint64_t au_desc = smem_desc_sw128(smem_u32(a_smem + stage * C::A_BYTES + BM * BK));
-          const uint64_t b_desc = smem_desc_sw128(smem_u32(b_smem + stage * C::B_BYTES));
+          const uint64_t a_desc = smem_desc_sw128(smem_u32(a_smem + stage * A_BYTES));
+          const uint64_t b_desc = smem_desc_sw128(smem_u32(b_smem + stage * B_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk) {
-            // +32 bytes per 32-element K step, in 16-byte units of the address field
+          for (int kk = 0; kk < BK / 32; ++kk)   // +32 bytes per K step = 2 in the address field
             umma_e4m3(d0, a_desc + 2 * kk, b_desc + 2 * kk, idesc, kk != 0);
-            if (GATED) umma_e4m3(d0 + BN, au_desc + 2 * kk, b_desc + 2 * kk, idesc, kk != 0);
-          }
           umma_commit(smem_u32(&empty[stage]));
           umma_commit(smem_u32(&pfull[pb]));
           any = true;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (any) {
         umma_commit(smem_u32(teardown));
-        mbar_wait_bounded(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
+        mbar_wait_sleep(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
       }
     }
     __syncwarp();
   } else {
+    regs_inc<kEpilogueRegs>();
     // ------------------------------------------------- promotion and epilogue
-    // Every epilogue warp walks the same tiles and, for gated tiles, passes one
-    // named barrier per tile whatever happens; after an expired wait it keeps
-    // walking with no further waits, loads or stores, so no barrier is missed.
-    const int ew = warp - 2;
+    // Thread = one activation row of the tile (its TMEM lane) and one half of
+    // the tile's columns.  Every epilogue warp walks the same tiles and K
+    // blocks and, for gated tiles, passes one named barrier per tile whatever
+    // happens: after an expired wait it keeps walking without further waits,
+    // loads or stores.
+    const int ew = warp - 4;              // 0..7
     const int q = warp & 3;               // TMEM lane quadrant
-    const int cq = ew >> 2;               // column quarter of the tile
-    const int c0 = cq * C::COLS;          // first tile column of this warp
+    const int hh = ew >> 2;               // column half
+    const int r = q * 32 + lane;          // row within the tile
     uint32_t kcount = 0;
     int tiles_done = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tiles_done) {
-      const Tile8 ti = decode_tile8<BN>(t, ts, go, p);
+      const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
       const bool routed = ti.g < p.E;
-      const int ncols = max(0, min(C::COLS, ti.n_mma - c0));   // multiple of 16
-      const float* sw = routed ? p.sa_routed + (size_t)ti.g * (p.rows_per_expert / BM) *
-                                                   ti.k_blocks
-                               : p.sa_shared;
-      const int rb_gate = ti.m;
-      const int rb_up = ((routed ? p.up_routed : p.up_shared) / BM) + ti.m;
-      float acc_g[C::COLS];
-      float acc_u[GATED ? C::COLS : 1];
+      const bool live = r < ti.nrows;
+      const bool any_cols = GATED || hh * 128 < ti.nfeat;
+      const int sw_kb = ti.k_blocks;
+      const float* sw = routed ? p.sw_routed + (size_t)ti.g * (p.rows_per_expert / 128) * sw_kb
+                               : p.sw_shared;
+      // weight scale rows: gated -> gate block and up block of f0; down -> block of this half
+      const int up = routed ? p.up_routed : p.up_shared;
+      const float* swa = sw + (size_t)((ti.f0 + (GATED ? 0 : hh * 128)) / 128) * sw_kb;
+      const float* swb = sw + (size_t)((up + ti.f0) / 128) * sw_kb;
+      const float* sa_row = p.sa + (size_t)(ti.row0 + r) * p.sa_ld;
+      float nxt_a = live ? sa_row[0] : 0.f;
+      float nxt_wa = swa[0];
+      float nxt_wb = GATED ? swb[0] : 0.f;
+
+      float acc_a[64], acc_b[64];        // gated: g and u of 64 features; down: 128 features
 #pragma unroll
-      for (int c = 0; c < C::COLS; ++c) acc_g[c] = 0.f;
-#pragma unroll
-      for (int c = 0; c < (GATED ? C::COLS : 1); ++c) acc_u[c] = 0.f;
-      for (int kb = 0; kb < ti.k_blocks && ok; ++kb, ++kcount) {
+      for (int c = 0; c < 64; ++c) { acc_a[c] = 0.f; acc_b[c] = 0.f; }
+      for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u;
         const uint32_t use = kcount >> 1;
-        if (!mbar_wait_bounded_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns, p.status,
-                                    p.timeout_bit)) {
-          ok = false;
-          break;
+        const float sa_cur = nxt_a;
+        const float s_a = nxt_wa * sa_cur;
+        const float s_b = (GATED ? nxt_wb : nxt_wa) * sa_cur;
+        if (kb + 1 < ti.k_blocks) {                   // next block's factors, fetched early
+          nxt_a = live ? sa_row[kb + 1] : 0.f;
+          nxt_wa = swa[kb + 1];
+          if (GATED) nxt_wb = swb[kb + 1];
         }
+        if (ok)
+          ok = mbar_wait_sleep_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns, p.status,
+                                    p.timeout_bit);
+        if (!ok) continue;
         tc_fence_after();
-        const float swg = sw[(size_t)rb_gate * ti.k_blocks + kb];
-        const float swu = GATED ? sw[(size_t)rb_up * ti.k_blocks + kb] : 0.f;
-        const float* sb = p.sb + (size_t)kb * p.R_cap + ti.row0 + c0;
-        const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride + c0;
+        if (any_cols) {
+          const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride;
+          float v[64];
+          if (GATED) {
+            // gate columns hh*64 .. +63 and up columns 128 + hh*64 .. +63
+            const uint32_t g0 = tl + hh * 64, u0 = tl + 128 + hh * 64;
+            tmem_ld_16x4(g0, g0 + 16, u0, u0 + 16, v);
 #pragma unroll
-        for (int cc = 0; cc < C::COLS; cc += 8) {
-          if (cc < ncols) {
-            float sa[8];
+            for (int c = 0; c < 32; ++c) acc_a[c] = fmaf(v[c], s_a, acc_a[c]);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) sa[c] = (c0 + cc + c < ti.nrows) ? sb[cc + c] : 0.f;
-            float v[8];
-            tmem_ld_8(tl + cc, v);
+            for (int c = 0; c < 32; ++c) acc_b[c] = fmaf(v[32 + c], s_b, acc_b[c]);
+            tmem_ld_16x4(g0 + 32, g0 + 48, u0 + 32, u0 + 48, v);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc_g[cc + c] = fmaf(v[c], swg * sa[c], acc_g[cc + c]);
-            if (GATED) {
-              tmem_ld_8(tl + BN + cc, v);
+            for (int c = 0; c < 32; ++c) acc_a[32 + c] = fmaf(v[c], s_a, acc_a[32 + c]);
 #pragma unroll
-              for (int c = 0; c < 8; ++c) acc_u[cc + c] = fmaf(v[c], swu * sa[c], acc_u[cc + c]);
-            }
+            for (int c = 0; c < 32; ++c) acc_b[32 + c] = fmaf(v[32 + c], s_b, acc_b[32 + c]);
+          } else {
+            // columns hh*128 .. +127, one weight scale block
+            const uint32_t c0 = tl + hh * 128;
+            tmem_ld_16x4(c0, c0 + 16, c0 + 32, c0 + 48, v);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) acc_a[c] = fmaf(v[c], s_a, acc_a[c]);
+            tmem_ld_16x4(c0 + 64, c0 + 80, c0 + 96, c0 + 112, v);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) acc_b[c] = fmaf(v[c], s_a, acc_b[c]);
           }
         }
         tc_fence_before();
@@ -317,41 +363,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(smem_u32(&pempty[pb]));
       }
 
-      const int feat = ti.m * BM + q * 32 + lane;     // output feature of this thread
       if (GATED) {
-        // h = silu(g) * u; one e4m3 scale per (row, the tile's 128 features)
-        float* red_p = red + (tiles_done & 1) * 4 * BN;          // [q][column]
+        // h = silu(g) * u over this thread's 64 features; the row's scale needs
+        // the max over both halves (the partner warp holds the other 64)
+        float amax = 0.f;
 #pragma unroll
-        for (int c = 0; c < C::COLS; ++c) {
-          const float g = acc_g[c];
-          const float h = g / (1.0f + __expf(-g)) * acc_u[c];
-          acc_g[c] = h;
-          float a = fabsf(h);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-          if (lane == 0) red_p[q * BN + c0 + c] = a;
+        for (int c = 0; c < 64; ++c) {
+          const float g = acc_a[c];
+          const float h = g / (1.0f + __expf(-g)) * acc_b[c];
+          acc_a[c] = h;
+          amax = fmaxf(amax, fabsf(h));
         }
-        named_bar_sync(1 + cq, 128);
-        if (ok) {
-          uint8_t* hq = static_cast<uint8_t*>(p.d);
+        float* red_p = red + (tiles_done & 1) * BMT * 2;
+        red_p[r * 2 + hh] = amax;
+        named_bar_sync(1, kEpiWarps * 32);
+        if (ok && live) {
+          const float m = fmaxf(red_p[r * 2], red_p[r * 2 + 1]);
+          const float s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+          const int row = ti.row0 + r;
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + (size_t)row * p.ldd +
+                                                ti.f0 + hh * 64);
 #pragma unroll
-          for (int c = 0; c < C::COLS; ++c) {
-            if (c < ncols && c0 + c < ti.nrows) {
-              const float amax = fmaxf(fmaxf(red_p[0 * BN + c0 + c], red_p[1 * BN + c0 + c]),
-                                       fmaxf(red_p[2 * BN + c0 + c], red_p[3 * BN + c0 + c]));
-              const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-              const int row = ti.row0 + c0 + c;
-              hq[(size_t)row * p.ldd + feat] = e4m3_of(__fdiv_rn(acc_g[c], s));
-              if (q == 0 && lane == 0) p.sd[(size_t)ti.m * p.R_cap + row] = s;
+          for (int w4 = 0; w4 < 4; ++w4) {
+            uint4 o;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = w4 * 16 + j * 4;
+              ow[j] = e4m3x4(__fdiv_rn(acc_a[c], s), __fdiv_rn(acc_a[c + 1], s),
+                             __fdiv_rn(acc_a[c + 2], s), __fdiv_rn(acc_a[c + 3], s));
             }
+            dst[w4] = o;
           }
+          if (hh == 0) p.sd[(size_t)row * (p.ldd / 128) + ti.f0 / 128] = s;
         }
-      } else if (ok) {
-        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d);
+      } else if (ok && live && any_cols) {
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(ti.row0 + r) * p.ldd +
+                           ti.f0 + hh * 128;
+        uint4* dst = reinterpret_cast<uint4*>(y);
 #pragma unroll
-        for (int c = 0; c < C::COLS; ++c)
-          if (c < ncols && c0 + c < ti.nrows)
-            y[(size_t)(ti.row0 + c0 + c) * p.ldd + feat] = __float2bfloat16_rn(acc_g[c]);
+        for (int w8 = 0; w8 < 16; ++w8) {
+          uint4 o;
+          __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = w8 * 8 + 2 * j;
+            const float a0 = c < 64 ? acc_a[c] : acc_b[c - 64];
+            const float a1 = c + 1 < 64 ? acc_a[c + 1] : acc_b[c + 1 - 64];
+            po[j] = __floats2bfloat162_rn(a0, a1);
+          }
+          dst[w8] = o;
+        }
       }
     }
   }
@@ -377,15 +439,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder8() {
   return fn;
 }
 
-// Row-major byte matrix [outer, inner] read in boxes of box_outer rows x 128
-// bytes, 128-byte swizzle, zero fill out of bounds.
-bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                 uint32_t box_outer) {
+// Row-major byte matrix [outer, inner] read in boxes of 128 rows x 128 bytes,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer) {
   auto enc = encoder8();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_outer};
+  cuuint32_t box[2] = {(cuuint32_t)BK, 128};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -393,30 +454,42 @@ bool make_map_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The register shares of the warpgroups only add up if the kernel was built
+// with exactly kLaunchRegs registers a thread; anything else is refused rather
+// than launched (a mismatched split would wait forever).
+template <bool GATED>
+cudaError_t check_register_split() {
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, grouped_gemm_fp8_kernel<GATED>);
+  if (e != cudaSuccess) return e;
+  return attr.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 }  // namespace
 
 cudaError_t prepare_grouped_gemm_fp8_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg8<true>::SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(grouped_gemm_fp8_kernel<false>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg8<false>::SMEM_BYTES);
+  cudaError_t e = check_register_split<true>();
+  if (e == cudaSuccess) e = check_register_split<false>();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  return e;
 }
 
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st) {
-  CUtensorMap tmA, tmAs, tmB;
+  CUtensorMap tmA, tmW, tmWs;
+  if (!make_map_u8(&tmA, a.b, a.K_ld, (uint64_t)a.R_cap)) return cudaErrorInvalidValue;
   const uint64_t rows_routed = (uint64_t)a.E * a.rows_per_expert;
-  if (!make_map_u8(&tmA, a.a_routed, a.K_routed, rows_routed, BM)) return cudaErrorInvalidValue;
+  if (!make_map_u8(&tmW, a.a_routed, a.K_routed, rows_routed)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
-    const uint64_t rows_shared = (uint64_t)a.m_tiles_shared * BM * (a.gated ? 2 : 1);
-    if (!make_map_u8(&tmAs, a.a_shared, a.K_shared, rows_shared, BM))
-      return cudaErrorInvalidValue;
+    const uint64_t rows_shared = a.gated ? (uint64_t)2 * a.up_shared : (uint64_t)a.feat_shared;
+    if (!make_map_u8(&tmWs, a.a_shared, a.K_shared, rows_shared)) return cudaErrorInvalidValue;
   } else {
-    tmAs = tmA;
+    tmWs = tmW;
   }
-  if (!make_map_u8(&tmB, a.b, a.K_ld, (uint64_t)a.R_cap, 16)) return cudaErrorInvalidValue;
 
   KParams8 p;
   p.group_offsets = a.group_offsets;
@@ -425,26 +498,27 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   p.kb_routed = a.K_routed / BK;
   p.kb_shared = a.K_shared / BK;
   p.rows_per_expert = a.rows_per_expert;
-  p.m_routed = a.m_tiles_routed;
-  p.m_shared = a.m_tiles_shared;
+  const int fpt = a.gated ? 128 : BNW;
+  p.feat_routed = a.feat_routed;
+  p.feat_shared = a.feat_shared;
+  p.ft_routed = (a.feat_routed + fpt - 1) / fpt;
+  p.ft_shared = (a.feat_shared + fpt - 1) / fpt;
   p.up_routed = a.up_routed;
   p.up_shared = a.up_shared;
-  p.sa_routed = a.sa_routed;
-  p.sa_shared = a.sa_shared != nullptr ? a.sa_shared : a.sa_routed;
-  p.sb = a.sb;
+  p.sw_routed = a.sa_routed;
+  p.sw_shared = a.sa_shared != nullptr ? a.sa_shared : a.sa_routed;
+  p.sa = a.sb;
+  p.sa_ld = a.K_ld / BK;
   p.d = a.d;
   p.sd = a.sd;
   p.ldd = a.ldd;
-  p.R_cap = a.R_cap;
   p.status = a.status;
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
   if (a.gated) {
-    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, Cfg8<true>::SMEM_BYTES, st>>>(
-        tmA, tmAs, tmB, p);
+    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
   } else {
-    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, Cfg8<false>::SMEM_BYTES, st>>>(
-        tmA, tmAs, tmB, p);
+    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
   }
   return cudaGetLastError();
 }

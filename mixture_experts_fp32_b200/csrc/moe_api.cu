@@ -37,6 +37,14 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+moe_status check_launch(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  g_last_cuda_error = e;
+  return MOE_ERR_CUDA;
+}
+
 moe_status ensure_device(moe_plan_s* p) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -50,8 +58,8 @@ moe_status ensure_device(moe_plan_s* p) {
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
   if (dev < 64 && !((prepared_mask >> dev) & 1ull)) {
-    if (moe::prepare_grouped_gemm_kernels() != cudaSuccess ||
-        moe::prepare_grouped_gemm_fp8_kernels() != cudaSuccess)
+    if (check_launch(moe::prepare_grouped_gemm_kernels()) != MOE_OK ||
+        check_launch(moe::prepare_grouped_gemm_fp8_kernels()) != MOE_OK)
       return MOE_ERR_CUDA;
     prepared_mask |= 1ull << dev;
   }
@@ -59,8 +67,6 @@ moe_status ensure_device(moe_plan_s* p) {
   p->device = dev;
   return MOE_OK;
 }
-
-moe_status check_launch(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 void record(moe_debug* dbg, int i, cudaStream_t st) {
   if (dbg != nullptr && dbg->events[i] != nullptr)
@@ -80,6 +86,10 @@ moe_status check_common(const moe_plan_s* p, int T, int k, const void* workspace
 }
 
 }  // namespace
+
+MOE_EXPORT const char* moe_last_cuda_error_string(void) {
+  return cudaGetErrorString(g_last_cuda_error);
+}
 
 MOE_EXPORT const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -310,8 +320,8 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
     fa.K_shared = H;
     fa.K_ld = H;
     fa.rows_per_expert = 2 * I;
-    fa.m_tiles_routed = I / 128;
-    fa.m_tiles_shared = S ? Is / 128 : 0;
+    fa.feat_routed = I;
+    fa.feat_shared = S ? Is : 0;
     fa.up_routed = I;
     fa.up_shared = Is;
     fa.ldd = plan->imax;
@@ -338,8 +348,8 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
     fa.K_shared = S ? Is : 0;
     fa.K_ld = plan->imax;
     fa.rows_per_expert = H;
-    fa.m_tiles_routed = H / 128;
-    fa.m_tiles_shared = S ? H / 128 : 0;
+    fa.feat_routed = H;
+    fa.feat_shared = S ? H : 0;
     fa.up_routed = 0;
     fa.up_shared = 0;
     fa.ldd = H;

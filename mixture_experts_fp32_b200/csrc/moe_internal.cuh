@@ -43,19 +43,19 @@ struct GroupedGemmArgs {
 // e4m3 grouped GEMM with one fp32 scale per 128x128 weight block and per 1x128
 // activation group (K blocks of 128).
 struct GroupedGemmFp8Args {
-  const void* a_routed;        // e4m3 [E * rows_per_expert, K_routed]
-  const void* a_shared;        // e4m3 [rows_shared, K_shared] or null
+  const void* a_routed;        // e4m3 weights [E * rows_per_expert, K_routed]
+  const void* a_shared;        // e4m3 weights [rows_shared, K_shared] or null
   const float* sa_routed;      // [E, rows_per_expert / 128, K_routed / 128]
   const float* sa_shared;      // [rows_shared / 128, K_shared / 128]
   const void* b;               // e4m3 activation rows [R_cap, K_ld]
-  const float* sb;             // their scales, transposed [K_ld / 128, R_cap]
+  const float* sb;             // their scales [R_cap, K_ld / 128]
   void* d;                     // gated: e4m3 h [R_cap, ldd]; down: bf16 y [R_cap, ldd]
-  float* sd;                   // gated: h scales, transposed [ldd / 128, R_cap]
+  float* sd;                   // gated: h scales [R_cap, ldd / 128]
   const int* group_offsets;
   int E, G;
   int K_routed, K_shared, K_ld;
   int rows_per_expert;
-  int m_tiles_routed, m_tiles_shared;
+  int feat_routed, feat_shared;   // output features of a group (gated: I, Is; down: H)
   int up_routed, up_shared;
   int ldd;
   int R_cap;
@@ -67,7 +67,7 @@ struct GroupedGemmFp8Args {
 };
 
 cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
-                                const int* total_rows, int R_cap, uint8_t* xq, float* sxT,
+                                const int* total_rows, int R_cap, uint8_t* xq, float* sx,
                                 int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st);
 cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
@@ -152,6 +152,53 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 >= limit_ns) {
       atomicOr(status, bit);
+      return false;
+    }
+  }
+}
+
+// try_wait that lets the hardware suspend the thread for up to hint_ns while
+// the phase is incomplete (it resumes when the phase completes), so waiting
+// warps do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 20000;
+
+// Bounded wait with suspension (single thread).
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity,
+                                                unsigned long long limit_ns,
+                                                unsigned int* status, unsigned int bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+    if (global_timer_ns() - t0 >= limit_ns) {
+      atomicOr(status, bit);
+      return false;
+    }
+  }
+}
+
+// Bounded wait with suspension taken by a whole warp (warp-uniform result).
+__device__ __forceinline__ bool mbar_wait_sleep_warp(uint32_t bar, uint32_t parity,
+                                                     unsigned long long limit_ns,
+                                                     unsigned int* status, unsigned int bit) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kSuspendHintNs))) return true;
+    if (__any_sync(0xffffffffu, global_timer_ns() - t0 >= limit_ns)) {
+      if ((threadIdx.x & 31) == 0) atomicOr(status, bit);
       return false;
     }
   }
@@ -247,6 +294,57 @@ __device__ __forceinline__ uint32_t idesc_e4m3_m128(int n) {
   return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute it).  The shares must add up to the registers the block was
+// launched with, or .inc waits forever: launchers check the kernel's register
+// count before launching.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// L2 eviction priority "normal" (operands reused by other tiles soon).
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// Four 16-column loads of this warp's lanes at four column offsets, one wait.
+__device__ __forceinline__ void tmem_ld_16x4(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, "
+      "%25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, "
+      "%41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%48, %49, %50, %51, %52, %53, %54, %55, %56, "
+      "%57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -259,30 +357,47 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       : "memory");
 }
 
+// Each thread of the warp reads 32 consecutive 32-bit columns of its own lane.
+// The load and its wait are one asm statement, so no use of the registers can
+// be scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld_32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Each thread of the warp reads 16 consecutive 32-bit columns of its own lane.
+// The load and its wait are one asm statement, so no use of the registers can
+// be scheduled before the data has arrived.
 __device__ __forceinline__ void tmem_ld_16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Each thread of the warp reads 8 consecutive 32-bit columns of its own lane.
+// The load and its wait are one asm statement, so no use of the registers can
+// be scheduled before the data has arrived.
 __device__ __forceinline__ void tmem_ld_8(uint32_t taddr, float (&v)[8]) {
   uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }

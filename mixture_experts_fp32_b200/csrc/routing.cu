@@ -226,14 +226,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
 
 // FP8 path: x_perm[r] = e4m3 codes of x[row_token[r]] with one scale per 1x128
 // group: s = amax / 448 (1 when amax = 0), q = e4m3_rne_sat(x / s), both fp32
-// divisions correctly rounded.  Scales are stored transposed, sxT[g][r], so
-// that a K block's scales for consecutive rows are contiguous.
+// divisions correctly rounded.  Scales are row-major, sx[r][g]: a GEMM thread
+// that owns row r reads its own row of scales.
 __global__ void __launch_bounds__(256) quant_gather_kernel(const __nv_bfloat16* __restrict__ x,
                                                            int H,
                                                            const int* __restrict__ row_token,
                                                            const int* __restrict__ total_rows,
                                                            int R_cap, uint8_t* __restrict__ xq,
-                                                           float* __restrict__ sxT) {
+                                                           float* __restrict__ sx) {
   const int R = *total_rows;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int groups = H / 128;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(256) quant_gather_kernel(const __nv_bfloat16* 
         packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
                   << (8 * i);
       *reinterpret_cast<uint32_t*>(xq + (size_t)r * H + (size_t)g * 128 + lane * 4) = packed;
-      if (lane == 0) sxT[(size_t)g * R_cap + r] = s;
+      if (lane == 0) sx[(size_t)r * groups + g] = s;
     }
   }
 }
@@ -299,12 +299,12 @@ cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, 
 }
 
 cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
-                                const int* total_rows, int R_cap, uint8_t* xq, float* sxT,
+                                const int* total_rows, int R_cap, uint8_t* xq, float* sx,
                                 int num_sms, cudaStream_t st) {
   int grid = num_sms * 8;
   if (grid > R_cap) grid = R_cap;
   if (grid < 1) grid = 1;
-  quant_gather_kernel<<<grid, 256, 0, st>>>(x, H, row_token, total_rows, R_cap, xq, sxT);
+  quant_gather_kernel<<<grid, 256, 0, st>>>(x, H, row_token, total_rows, R_cap, xq, sx);
   return cudaGetLastError();
 }
 

@@ -58,7 +58,6 @@ def test_fp8_activation_codes_bit_exact():
     v = plan.views()
     torch.cuda.synchronize()
     R = int(res["offsets"][-1]) + w.T
-    C = w.T * (w.k + w.S)
 
     def dev_view(ptr, n, dtype):
         off = ptr - plan.workspace.data_ptr()
@@ -67,9 +66,9 @@ def test_fp8_activation_codes_bit_exact():
 
     rowtok = dev_view(v.row_token, R, torch.int32).numpy()
     codes = dev_view(v.x_perm, R * w.H, torch.uint8).numpy().reshape(R, w.H)
-    scales = dev_view(v.x_scale, (w.H // 128) * C, torch.float32).numpy().reshape(w.H // 128, C)
+    scales = dev_view(v.x_scale, R * (w.H // 128), torch.float32).numpy().reshape(R, w.H // 128)
     xf = oracle.bf16_to_f64(inp["x"]).reshape(w.T, w.H).astype(np.float32)
     for r in range(R):
         q, s = oracle.quant_row_e4m3(xf[rowtok[r]])
         assert np.array_equal(codes[r], q), r
-        assert np.array_equal(scales[:, r], s), r
+        assert np.array_equal(scales[r], s), r
