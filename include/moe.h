@@ -70,6 +70,7 @@ typedef enum {
 #define MOE_DEV_WAIT_TIMEOUT_GATE_UP 0x1u   /* a bounded wait expired in the gate/up GEMM */
 #define MOE_DEV_WAIT_TIMEOUT_DOWN    0x2u   /* a bounded wait expired in the down GEMM */
 #define MOE_DEV_BAD_EXPERT_ID        0x4u   /* a routed expert index outside [0, E) */
+#define MOE_DEV_WAIT_TIMEOUT_ROUTER  0x8u   /* a bounded wait expired in the router GEMM */
 
 /* Shape of the layer; fixed for the lifetime of a plan. */
 typedef struct {

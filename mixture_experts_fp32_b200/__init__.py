@@ -26,6 +26,7 @@ MOE_W_FP8_E4M3_B128 = 1
 MOE_DEV_WAIT_TIMEOUT_GATE_UP = 0x1
 MOE_DEV_WAIT_TIMEOUT_DOWN = 0x2
 MOE_DEV_BAD_EXPERT_ID = 0x4
+MOE_DEV_WAIT_TIMEOUT_ROUTER = 0x8
 
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")

@@ -9,8 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["moe_api.cu", "router.cu", "routing.cu", "grouped_gemm.cu", "grouped_gemm_fp8.cu",
-           "noalloc.cu"]
+SOURCES = ["moe_api.cu", "router_tc.cu", "topk.cu", "routing.cu", "grouped_gemm.cu",
+           "grouped_gemm_fp8.cu", "noalloc.cu"]
 HEADERS = ["moe_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -17,8 +17,8 @@ struct moe_plan_s {
   int ks_max;        // top_k_max + S
   size_t r_cap;      // max_tokens * ks_max rows
   // byte offsets inside the workspace
-  size_t off_status, off_goff, off_partial, off_logits, off_ids, off_w, off_perm, off_inv,
-      off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
+  size_t off_status, off_goff, off_wsplit, off_partial, off_logits, off_ids, off_w, off_perm,
+      off_inv, off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
   unsigned long long wait_limit_ns;
   int device;
   int num_sms;
@@ -59,7 +59,8 @@ moe_status ensure_device(moe_plan_s* p) {
   if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;   // built for sm_100a only
   if (dev < 64 && !((prepared_mask >> dev) & 1ull)) {
     if (check_launch(moe::prepare_grouped_gemm_kernels()) != MOE_OK ||
-        check_launch(moe::prepare_grouped_gemm_fp8_kernels()) != MOE_OK)
+        check_launch(moe::prepare_grouped_gemm_fp8_kernels()) != MOE_OK ||
+        check_launch(moe::prepare_router_kernel()) != MOE_OK)
       return MOE_ERR_CUDA;
     prepared_mask |= 1ull << dev;
   }
@@ -140,6 +141,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   };
   p->off_status = take(64);
   p->off_goff = take(sizeof(int) * (E + 2));
+  p->off_wsplit = take(2 * 3 * (size_t)moe::router_padded_experts((int)E) * H);
   p->off_partial = take(sizeof(float) * moe::kRouterSplitMax * T * E);
   p->off_logits = take(sizeof(float) * T * E);
   p->off_ids = take(sizeof(int) * T * c.top_k_max);
@@ -226,10 +228,11 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
 
   record(dbg, 0, st);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
-  int splits = 1, kchunk = H;
-  moe::router_split_plan(T, E, H, plan->num_sms, &splits, &kchunk);
-  s = check_launch(moe::launch_router_logits(x, valid, T, H, wts->router_w, E, partial, splits,
-                                             kchunk, st));
+  int splits = 1, kb_per_split = H / 64;
+  moe::router_split_plan(T, E, H, plan->num_sms, &splits, &kb_per_split);
+  s = check_launch(moe::launch_router_logits_tc(
+      x, valid, T, H, wts->router_w, E, at<__nv_bfloat16>(workspace, plan->off_wsplit), partial,
+      splits, kb_per_split, plan->num_sms, status, st));
   if (s != MOE_OK) return s;
   record(dbg, 1, st);
   s = check_launch(moe::launch_topk(partial, splits, wts->router_b, valid, T, E, k, c.renormalize,
