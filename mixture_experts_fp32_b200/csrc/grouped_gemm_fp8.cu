@@ -312,9 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float nxt_wa = swa[0];
       float nxt_wb = GATED ? swb[0] : 0.f;
 
-      float acc_a[64], acc_b[64];        // gated: g and u of 64 features; down: 128 features
+      // gated: g and u of 64 features; down: 128 features.  Pairs of columns
+      // are updated by one packed fp32 FMA (same rounding as two scalar FMAs).
+      float2 acc_a[32], acc_b[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) { acc_a[c] = 0.f; acc_b[c] = 0.f; }
+      for (int c = 0; c < 32; ++c) {
+        acc_a[c] = make_float2(0.f, 0.f);
+        acc_b[c] = make_float2(0.f, 0.f);
+      }
       for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u;
         const uint32_t use = kcount >> 1;
@@ -331,48 +336,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     p.timeout_bit);
         if (!ok) continue;
         tc_fence_after();
+        // the partial buffer goes back to the MMA as soon as it has been read
+        auto release = [&]() {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&pempty[pb]));
+        };
         if (any_cols) {
           const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride;
           float v[64];
+          const float2 sa2 = make_float2(s_a, s_a), sb2 = make_float2(s_b, s_b);
           if (GATED) {
             // gate columns hh*64 .. +63 and up columns 128 + hh*64 .. +63
             const uint32_t g0 = tl + hh * 64, u0 = tl + 128 + hh * 64;
             tmem_ld_16x4(g0, g0 + 16, u0, u0 + 16, v);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc_a[c] = fmaf(v[c], s_a, acc_a[c]);
+            for (int c = 0; c < 16; ++c)
+              acc_a[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[c]);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc_b[c] = fmaf(v[32 + c], s_b, acc_b[c]);
+            for (int c = 0; c < 16; ++c)
+              acc_b[c] = __ffma2_rn(make_float2(v[32 + 2 * c], v[33 + 2 * c]), sb2, acc_b[c]);
             tmem_ld_16x4(g0 + 32, g0 + 48, u0 + 32, u0 + 48, v);
+            release();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc_a[32 + c] = fmaf(v[c], s_a, acc_a[32 + c]);
+            for (int c = 0; c < 16; ++c)
+              acc_a[16 + c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[16 + c]);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc_b[32 + c] = fmaf(v[32 + c], s_b, acc_b[32 + c]);
+            for (int c = 0; c < 16; ++c)
+              acc_b[16 + c] =
+                  __ffma2_rn(make_float2(v[32 + 2 * c], v[33 + 2 * c]), sb2, acc_b[16 + c]);
           } else {
             // columns hh*128 .. +127, one weight scale block
             const uint32_t c0 = tl + hh * 128;
             tmem_ld_16x4(c0, c0 + 16, c0 + 32, c0 + 48, v);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) acc_a[c] = fmaf(v[c], s_a, acc_a[c]);
+            for (int c = 0; c < 32; ++c)
+              acc_a[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[c]);
             tmem_ld_16x4(c0 + 64, c0 + 80, c0 + 96, c0 + 112, v);
+            release();
 #pragma unroll
-            for (int c = 0; c < 64; ++c) acc_b[c] = fmaf(v[c], s_a, acc_b[c]);
+            for (int c = 0; c < 32; ++c)
+              acc_b[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_b[c]);
           }
+        } else {
+          release();
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&pempty[pb]));
       }
 
       if (GATED) {
         // h = silu(g) * u over this thread's 64 features; the row's scale needs
         // the max over both halves (the partner warp holds the other 64)
         float amax = 0.f;
+        float hv[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float g = acc_a[c];
-          const float h = g / (1.0f + __expf(-g)) * acc_b[c];
-          acc_a[c] = h;
-          amax = fmaxf(amax, fabsf(h));
+          const float g = (c & 1) ? acc_a[c >> 1].y : acc_a[c >> 1].x;
+          const float u = (c & 1) ? acc_b[c >> 1].y : acc_b[c >> 1].x;
+          hv[c] = g / (1.0f + __expf(-g)) * u;
+          amax = fmaxf(amax, fabsf(hv[c]));
         }
         float* red_p = red + (tiles_done & 1) * BMT * 2;
         red_p[r * 2 + hh] = amax;
@@ -390,8 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int c = w4 * 16 + j * 4;
-              ow[j] = e4m3x4(__fdiv_rn(acc_a[c], s), __fdiv_rn(acc_a[c + 1], s),
-                             __fdiv_rn(acc_a[c + 2], s), __fdiv_rn(acc_a[c + 3], s));
+              ow[j] = e4m3x4(__fdiv_rn(hv[c], s), __fdiv_rn(hv[c + 1], s),
+                             __fdiv_rn(hv[c + 2], s), __fdiv_rn(hv[c + 3], s));
             }
             dst[w4] = o;
           }
@@ -407,10 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int c = w8 * 8 + 2 * j;
-            const float a0 = c < 64 ? acc_a[c] : acc_b[c - 64];
-            const float a1 = c + 1 < 64 ? acc_a[c + 1] : acc_b[c + 1 - 64];
-            po[j] = __floats2bfloat162_rn(a0, a1);
+            const int c2 = w8 * 4 + j;                 // column pair
+            const float2 a = c2 < 32 ? acc_a[c2] : acc_b[c2 - 32];
+            po[j] = __floats2bfloat162_rn(a.x, a.y);
           }
           dst[w8] = o;
         }

@@ -17,8 +17,9 @@ struct moe_plan_s {
   int ks_max;        // top_k_max + S
   size_t r_cap;      // max_tokens * ks_max rows
   // byte offsets inside the workspace
-  size_t off_status, off_goff, off_wsplit, off_partial, off_logits, off_ids, off_w, off_perm,
-      off_inv, off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
+  size_t off_status, off_goff, off_wsplit, off_rscratch, off_partial, off_logits, off_ids, off_w,
+      off_perm,
+      off_inv, off_rowtok, off_xp, off_sx, off_xqt, off_sxt, off_h, off_sh, off_y;
   unsigned long long wait_limit_ns;
   int device;
   int num_sms;
@@ -142,6 +143,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   p->off_status = take(64);
   p->off_goff = take(sizeof(int) * (E + 2));
   p->off_wsplit = take(2 * 3 * (size_t)moe::router_padded_experts((int)E) * H);
+  p->off_rscratch = take(sizeof(int) * (size_t)moe::route_scratch_ints((int)T, (int)E));
   p->off_partial = take(sizeof(float) * moe::kRouterSplitMax * T * E);
   p->off_logits = take(sizeof(float) * T * E);
   p->off_ids = take(sizeof(int) * T * c.top_k_max);
@@ -152,7 +154,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   if (c.wtype == MOE_W_BF16) {
     // bf16 permuted rows and h; fp32 expert outputs
     p->off_xp = take(2 * r_cap * H);
-    p->off_sx = 0;
+    p->off_sx = p->off_xqt = p->off_sxt = 0;
     p->off_h = take(2 * r_cap * (size_t)imax);
     p->off_sh = 0;
     p->off_y = take(sizeof(float) * r_cap * H);
@@ -160,6 +162,8 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
     // e4m3 permuted rows and h with transposed 1x128 scales; bf16 expert outputs
     p->off_xp = take(r_cap * H);
     p->off_sx = take(sizeof(float) * (H / 128) * r_cap);
+    p->off_xqt = take(T * H);                             // each token quantised once
+    p->off_sxt = take(sizeof(float) * (H / 128) * T);
     p->off_h = take(r_cap * (size_t)imax);
     p->off_sh = take(sizeof(float) * ((size_t)imax / 128) * r_cap);
     p->off_y = take(2 * r_cap * H);
@@ -239,7 +243,8 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
                                     logits, ids, w, st));
   if (s != MOE_OK) return s;
   record(dbg, 2, st);
-  s = check_launch(moe::launch_route(ids, valid, T, E, k, S, goff, perm, inv, rowtok, status, st));
+  s = check_launch(moe::launch_route(ids, valid, T, E, k, S, goff, perm, inv, rowtok, status,
+                                     at<int>(workspace, plan->off_rscratch), st));
   if (s != MOE_OK) return s;
   record(dbg, 3, st);
   const bool fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
@@ -247,10 +252,10 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
     s = check_launch(
         moe::launch_gather_rows(x, H, rowtok, goff + G, R_cap, xp, plan->num_sms, st));
   } else {
-    s = check_launch(moe::launch_quant_gather(x, H, rowtok, goff + G, R_cap,
-                                              at<uint8_t>(workspace, plan->off_xp),
-                                              at<float>(workspace, plan->off_sx), plan->num_sms,
-                                              st));
+    s = check_launch(moe::launch_quant_gather(
+        x, valid, T, H, rowtok, goff + G, R_cap, at<uint8_t>(workspace, plan->off_xqt),
+        at<float>(workspace, plan->off_sxt), at<uint8_t>(workspace, plan->off_xp),
+        at<float>(workspace, plan->off_sx), plan->num_sms, st));
   }
   if (s != MOE_OK) return s;
   record(dbg, 4, st);
@@ -407,7 +412,8 @@ MOE_EXPORT moe_status moe_route_from_logits(moe_plan_t plan, const float* logits
   if (s != MOE_OK) return s;
   s = check_launch(moe::launch_route(topk_ids, valid, T, E, k, S, goff, perm,
                                      at<int>(workspace, plan->off_inv),
-                                     at<int>(workspace, plan->off_rowtok), status, st));
+                                     at<int>(workspace, plan->off_rowtok), status,
+                                     at<int>(workspace, plan->off_rscratch), st));
   if (s != MOE_OK) return s;
   if (cudaMemcpyAsync(offsets, goff, sizeof(int) * (E + 1), cudaMemcpyDeviceToDevice, st) !=
       cudaSuccess)

@@ -66,8 +66,11 @@ struct GroupedGemmFp8Args {
   int num_ctas;
 };
 
-cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
-                                const int* total_rows, int R_cap, uint8_t* xq, float* sx,
+// FP8: quantise every valid token once (xq_tok [T, H], sx_tok [T, H/128]), then
+// copy codes and scales into permuted order (xp [R, H], sxp [R, H/128]).
+cudaError_t launch_quant_gather(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
+                                const int* row_token, const int* total_rows, int R_cap,
+                                uint8_t* xq_tok, float* sx_tok, uint8_t* xp, float* sxp,
                                 int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st);
 cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
@@ -86,9 +89,12 @@ cudaError_t prepare_router_kernel();
 cudaError_t launch_topk(const float* partial, int splits, const float* bias, const uint8_t* valid,
                         int T, int E, int k, int renorm, float* logits_out, int* ids, float* w,
                         cudaStream_t st);
+// scratch: route_scratch_ints(T, E) ints for batches of more than 1024 tokens
+// (parallel chunks); nullptr runs the single-block kernel.
+int route_scratch_ints(int max_tokens, int E);
 cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int k, int S,
                          int* group_offsets, int* perm, int* inv, int* row_token,
-                         unsigned int* status, cudaStream_t st);
+                         unsigned int* status, int* scratch, cudaStream_t st);
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_token,
                                const int* total_rows, int R_cap, __nv_bfloat16* xp,
                                int num_sms, cudaStream_t st);

@@ -77,7 +77,8 @@ MOE_EXPORT moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float
     return MOE_ERR_CUDA;
   if (moe::launch_route(topk_ids, valid, T, (int)E, k, (int)S, goff, perm,
                         reinterpret_cast<int*>(scratch + off_inv),
-                        reinterpret_cast<int*>(scratch + off_rowtok), status, st) != cudaSuccess)
+                        reinterpret_cast<int*>(scratch + off_rowtok), status, nullptr,
+                        st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (cudaMemcpyAsync(offsets, goff, sizeof(int) * (E + 1), cudaMemcpyDeviceToDevice, st) !=
       cudaSuccess)

@@ -148,6 +148,128 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
   }
 }
 
+// The same permutation for many chunks in parallel: (1) each chunk counts its
+// pairs per expert and its valid tokens, (2) one block turns the counts into
+// group offsets and per-chunk bases (expert-major, chunk-minor, so tokens stay
+// ascending inside an expert), (3) each chunk ranks and scatters its pairs.
+// Identical results to route_kernel.
+__global__ void __launch_bounds__(1024, 1) route_count_kernel(const int* __restrict__ ids,
+                                                              const uint8_t* __restrict__ valid,
+                                                              int T, int E, int k,
+                                                              int* __restrict__ chunk_cnt,
+                                                              int* __restrict__ chunk_valid,
+                                                              unsigned int* status) {
+  __shared__ uint32_t bits[kMaxExperts][32];
+  __shared__ int wvalid[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, c = blockIdx.x;
+  for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
+  __syncthreads();
+  const int t = c * kChunk + tid;
+  set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+  const uint32_t vb = __ballot_sync(0xffffffffu, t < T && (valid == nullptr || valid[t]));
+  if (lane == 0) wvalid[warp] = __popc(vb);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int s = 0;
+    for (int w = 0; w < 32; ++w) s += __popc(bits[e][w]);
+    chunk_cnt[(size_t)c * E + e] = s;
+  }
+  if (tid == 0) {
+    int s = 0;
+    for (int w = 0; w < 32; ++w) s += wvalid[w];
+    chunk_valid[c] = s;
+  }
+}
+
+__global__ void __launch_bounds__(1024, 1) route_scan_kernel(const int* __restrict__ chunk_cnt,
+                                                             const int* __restrict__ chunk_valid,
+                                                             int nchunks, int E, int S,
+                                                             int* __restrict__ chunk_base,
+                                                             int* __restrict__ vbase,
+                                                             int* __restrict__ group_offsets) {
+  __shared__ int tot[kMaxExperts];
+  __shared__ int s_valid;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int s = 0;
+    for (int c = 0; c < nchunks; ++c) s += chunk_cnt[(size_t)c * E + e];
+    tot[e] = s;
+  }
+  if (tid == 0) {
+    int s = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      vbase[c] = s;
+      s += chunk_valid[c];
+    }
+    s_valid = s;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      const int v = tot[e];
+      tot[e] = acc;
+      group_offsets[e] = acc;
+      acc += v;
+    }
+    group_offsets[E] = acc;
+    if (S) group_offsets[E + 1] = acc + s_valid;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = tot[e];
+    for (int c = 0; c < nchunks; ++c) {
+      chunk_base[(size_t)c * E + e] = run;
+      run += chunk_cnt[(size_t)c * E + e];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
+    const int* __restrict__ ids, const uint8_t* __restrict__ valid, int T, int E, int k, int S,
+    const int* __restrict__ chunk_base, const int* __restrict__ vbase,
+    const int* __restrict__ group_offsets, int* __restrict__ perm, int* __restrict__ inv,
+    int* __restrict__ row_token, unsigned int* status) {
+  __shared__ uint32_t bits[kMaxExperts][32];
+  __shared__ int wvalid[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, c = blockIdx.x;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
+  __syncthreads();
+  const int t = c * kChunk + tid;
+  set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+  const bool ok = t < T && (valid == nullptr || valid[t]);
+  const uint32_t vb = __ballot_sync(0xffffffffu, ok);
+  if (lane == 0) wvalid[warp] = __popc(vb);
+  __syncthreads();
+  if (t >= T) return;
+  const int ks = k + S;
+  if (!ok) {
+    for (int j = 0; j < ks; ++j) inv[(size_t)t * ks + j] = -1;
+    return;
+  }
+  for (int j = 0; j < k; ++j) {
+    const int e = ids[(size_t)t * k + j];
+    if (e < 0 || e >= E) {
+      inv[(size_t)t * ks + j] = -1;
+      continue;
+    }
+    int r = chunk_base[(size_t)c * E + e];
+    for (int w = 0; w < warp; ++w) r += __popc(bits[e][w]);
+    r += __popc(bits[e][warp] & lt_mask);
+    perm[r] = t * k + j;
+    inv[(size_t)t * ks + j] = r;
+    row_token[r] = t;
+  }
+  if (S) {
+    int vr = vbase[c] + __popc(vb & lt_mask);
+    for (int w = 0; w < warp; ++w) vr += wvalid[w];
+    const int pos = group_offsets[E] + vr;
+    inv[(size_t)t * ks + k] = pos;
+    row_token[pos] = t;
+  }
+}
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                           int H,
                                                           const int* __restrict__ row_token,
@@ -224,49 +346,92 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
   }
 }
 
-// FP8 path: x_perm[r] = e4m3 codes of x[row_token[r]] with one scale per 1x128
-// group: s = amax / 448 (1 when amax = 0), q = e4m3_rne_sat(x / s), both fp32
-// divisions correctly rounded.  Scales are row-major, sx[r][g]: a GEMM thread
-// that owns row r reads its own row of scales.
-__global__ void __launch_bounds__(256) quant_gather_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           int H,
-                                                           const int* __restrict__ row_token,
-                                                           const int* __restrict__ total_rows,
-                                                           int R_cap, uint8_t* __restrict__ xq,
+// FP8 path, activation quantisation of each valid token once: e4m3 codes of
+// x[t] with one scale per 1x128 group, s = amax / 448 (1 when amax = 0),
+// q = e4m3_rne_sat(x / s), both fp32 divisions correctly rounded.  A warp owns
+// one group (4 values a lane).  Scales are row-major, sx[t][g].
+__global__ void __launch_bounds__(256) quant_tokens_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           const uint8_t* __restrict__ valid,
+                                                           int T, int H,
+                                                           uint8_t* __restrict__ xq,
                                                            float* __restrict__ sx) {
-  const int R = *total_rows;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int groups = H / 128;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long wg = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+       wg < (long long)T * groups; wg += nwarps) {
+    const int t = (int)(wg / groups), g = (int)(wg - (long long)t * groups);
+    if (valid != nullptr && !valid[t]) continue;
+    const uint2 raw =
+        *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)g * 128 + lane * 4);
+    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
+    float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
+                << (8 * i);
+    *reinterpret_cast<uint32_t*>(xq + (size_t)t * H + (size_t)g * 128 + lane * 4) = packed;
+    if (lane == 0) sx[(size_t)t * groups + g] = s;
+  }
+}
+
+// x_perm[r] = xq[row_token[r]] and its scale row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_fp8_rows_kernel(const uint8_t* __restrict__ xq,
+                                                              const float* __restrict__ sx,
+                                                              int H,
+                                                              const int* __restrict__ row_token,
+                                                              const int* __restrict__ total_rows,
+                                                              uint8_t* __restrict__ xp,
+                                                              float* __restrict__ sxp) {
+  const int R = *total_rows;
+  const int nv = H / 16, groups = H / 128;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     const int t = row_token[r];
-    for (int g = warp; g < groups; g += blockDim.x / 32) {
-      const uint2 raw =
-          *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)g * 128 + lane * 4);
-      const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-      const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-      const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
-      float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-      const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-      uint32_t packed = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
-                  << (8 * i);
-      *reinterpret_cast<uint32_t*>(xq + (size_t)r * H + (size_t)g * 128 + lane * 4) = packed;
-      if (lane == 0) sx[(size_t)r * groups + g] = s;
-    }
+    const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * H);
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) dst[v] = src[v];
+    for (int g = threadIdx.x; g < groups; g += blockDim.x)
+      sxp[(size_t)r * groups + g] = sx[(size_t)t * groups + g];
   }
 }
 
 }  // namespace
 
+int route_scratch_ints(int max_tokens, int E) {
+  const int nchunks = (max_tokens + kChunk - 1) / kChunk;
+  return nchunks * (2 * E + 2);
+}
+
 cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int k, int S,
                          int* group_offsets, int* perm, int* inv, int* row_token,
-                         unsigned int* status, cudaStream_t st) {
-  route_kernel<<<1, 1024, 0, st>>>(ids, valid, T, E, k, S, group_offsets, perm, inv, row_token,
-                                   status);
+                         unsigned int* status, int* scratch, cudaStream_t st) {
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  if (nchunks <= 1 || scratch == nullptr) {
+    route_kernel<<<1, 1024, 0, st>>>(ids, valid, T, E, k, S, group_offsets, perm, inv, row_token,
+                                     status);
+    return cudaGetLastError();
+  }
+  int* chunk_cnt = scratch;                        // [nchunks][E]
+  int* chunk_base = chunk_cnt + (size_t)nchunks * E;   // [nchunks][E]
+  int* chunk_valid = chunk_base + (size_t)nchunks * E; // [nchunks]
+  int* vbase = chunk_valid + nchunks;                  // [nchunks]
+  route_count_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, chunk_cnt, chunk_valid,
+                                               status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  route_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, chunk_valid, nchunks, E, S, chunk_base, vbase,
+                                        group_offsets);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // set_bits reports a bad expert id once in the count pass; the scatter pass skips it quietly
+  route_scatter_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, S, chunk_base, vbase,
+                                                 group_offsets, perm, inv, row_token, status);
   return cudaGetLastError();
 }
 
@@ -298,13 +463,20 @@ cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_gather(const __nv_bfloat16* x, int H, const int* row_token,
-                                const int* total_rows, int R_cap, uint8_t* xq, float* sx,
+cudaError_t launch_quant_gather(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
+                                const int* row_token, const int* total_rows, int R_cap,
+                                uint8_t* xq_tok, float* sx_tok, uint8_t* xp, float* sxp,
                                 int num_sms, cudaStream_t st) {
+  const long long warps = (long long)T * (H / 128);
+  long long g1 = (warps + 7) / 8;
+  if (g1 > (long long)num_sms * 16) g1 = (long long)num_sms * 16;
+  quant_tokens_kernel<<<(int)g1, 256, 0, st>>>(x, valid, T, H, xq_tok, sx_tok);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   int grid = num_sms * 8;
   if (grid > R_cap) grid = R_cap;
   if (grid < 1) grid = 1;
-  quant_gather_kernel<<<grid, 256, 0, st>>>(x, H, row_token, total_rows, R_cap, xq, sx);
+  gather_fp8_rows_kernel<<<grid, 256, 0, st>>>(xq_tok, sx_tok, H, row_token, total_rows, xp, sxp);
   return cudaGetLastError();
 }
 
