@@ -14,36 +14,51 @@
 // fp32 register accumulators with its scale ("promotion").  Two partial
 // buffers let the tensor core run one K block ahead of the promotion.
 //
-// Rows of activations take the MMA's M side (128 per tile) and weight rows its
-// N side (256): a TMEM lane is one activation row, so the activation scale of a
-// K block is one register per thread and the weight scale one per 128 columns;
-// promotion is one FMA per value, and each thread writes its row contiguously.
+// CTA pairs.  A tile is 256 activation rows x 256 weight rows, computed by the
+// two CTAs of a cluster with cta_group::2 MMAs (M = 256, N = 256): each CTA
+// stages its own 128 activation rows and one half (128 rows) of the weight
+// tile, and receives its 128 rows x all 256 columns in its own tensor memory.
+// Per 128-K block a CTA moves 32 KB through shared memory instead of the 48 KB
+// of a one-CTA 128 x 256 tile, and shared-memory bandwidth (TMA writes plus
+// tensor-core operand reads) is what bounds a one-CTA e4m3 tile on sm_100.
+// The even CTA of the pair issues the MMAs and owns the stage barriers: both
+// CTAs' TMA loads complete their bytes on it (cta_group::2 form of the load),
+// and the odd CTA's epilogue warps return partial buffers to it by remote
+// mbarrier arrivals.  No load is multicast.
 //
-//   gated: a tile owns 128 features of h for up to 128 rows of one group: the
-//          B operand stacks the matching 128 gate rows and 128 up rows (N = 256),
-//          so g and u of a feature sit in the same TMEM lane.  After the last K
+// Rows of activations take the MMA's M side and weight rows its N side: a TMEM
+// lane is one activation row, so the activation scale of a K block is one
+// register per thread and the weight scale one per 128 columns; promotion is
+// one FMA per value, and each thread writes its row contiguously.
+//
+//   gated: a pair tile owns 128 features of h: the even CTA stages their 128
+//          gate rows, the odd CTA their 128 up rows (N = 256), so g and u of a
+//          feature sit in the same TMEM lane of both CTAs.  After the last K
 //          block h = silu(g) * u is quantised per 1x128 group (the tile's 128
 //          features are one group) into e4m3 codes and an fp32 scale.
-//   down:  a tile owns up to 256 output features (two weight scale blocks) for
-//          up to 128 rows; y is written in bf16.
+//   down:  a pair tile owns 256 output features (two weight scale blocks, one
+//          staged by each CTA); y is written in bf16.
 //
 // Three warpgroups (384 threads).  Warpgroup 0: warp 0 issues TMA loads, warp 1
-// owns tensor memory and issues the MMAs; it gives registers back
-// (setmaxnreg.dec).  Warpgroups 1 and 2 (8 warps) promote and finish, with the
-// registers warpgroup 0 released: warp w reads TMEM lanes 32*(w%4)... and one
-// half of the tile's columns, 128 fp32 accumulators a thread.  Every wait is
-// bounded and suspends rather than spins.
+// owns tensor memory and, in the even CTA, issues the MMAs; it gives registers
+// back (setmaxnreg.dec).  Warpgroups 1 and 2
+// (8 warps) promote and finish, with the registers warpgroup 0 released: warp w
+// reads TMEM lanes 32*(w%4)... and one half of the tile's columns, 128 fp32
+// accumulators a thread.  Every wait is bounded and suspends rather than spins.
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int BMT = 128;           // activation rows per tile (MMA M)
+constexpr int BMT = 128;           // activation rows per CTA (a pair covers 2 * BMT)
+constexpr int PAIR_ROWS = 2 * BMT;
 constexpr int BK = 128;            // e4m3 elements (= bytes) per K block: one scale group
-constexpr int BNW = 256;           // weight rows per tile (MMA N)
+constexpr int BNW = 256;           // weight rows per pair tile (MMA N); 128 staged per CTA
 constexpr int kEpiWarps = 8;       // two per TMEM lane quadrant, each half of the columns
 constexpr int kThreads = 384;
 // 12 warps leave each SM sub-partition three warps: 168 registers a thread at
@@ -57,13 +72,135 @@ static_assert(128 * kProducerRegs + 256 * kEpilogueRegs == kThreads * kLaunchReg
               "register shares must add up to the launch's registers");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPartStride = 256;   // TMEM columns between the two partial buffers
-constexpr int A_BYTES = BMT * BK;  // 16 KB
-constexpr int B_BYTES = BNW * BK;  // 32 KB
-constexpr int STAGES = 4;
+constexpr int A_BYTES = BMT * BK;              // 16 KB: this CTA's activation rows
+constexpr int B_BYTES = (BNW / 2) * BK;        // 16 KB: this CTA's half of the weight rows
+constexpr int STAGES = 6;
 constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
 constexpr int RED_BYTES = 2 * BMT * 2 * 4;    // h amax halves [tile parity][row][half]
 constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 2048;
 constexpr unsigned long long kTeardownLimitNs = 1000000000ull;
+
+// ------------------------------------------------------- CTA-pair primitives
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+// Remote arrival that publishes no memory: returning a tensor-memory partial
+// buffer, whose reads tcgen05.wait::ld has already completed and
+// tcgen05.fence::before_thread_sync has ordered before this arrival.  A
+// cluster-scope release here would cost a cluster-wide fence on the MMA's
+// critical path.
+__device__ __forceinline__ void mbar_arrive_remote_signal(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 2-D tiled TMA load (no multicast) into this CTA's shared memory whose bytes
+// complete on an mbarrier of either CTA of the pair (here: the even CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int x, int y,
+                                                 uint32_t bar_cluster, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cluster), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256.
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the mbarrier at this shared-memory offset in both CTAs of the pair
+// once the pair MMAs this thread issued so far have completed.
+__device__ __forceinline__ void umma_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"((uint16_t)0x3)
+      : "memory");
+}
+// kind::f8f6f4 instruction descriptor for M = 256, N = 256, e4m3 x e4m3 -> f32.
+constexpr uint32_t kIdescPair = (1u << 4) | ((uint32_t)(BNW >> 3) << 17) |
+                                ((uint32_t)(PAIR_ROWS >> 4) << 24);
+
+// A scale fetched ahead of its use: the asm keeps the load where it is written
+// (the compiler may not sink it next to the use and expose its latency).
+__device__ __forceinline__ float ldg_ahead(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
+// Two 16-column TMEM loads without a wait, and the wait that ties the
+// registers: no use of r can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_2x16(uint32_t a0, uint32_t a1, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, "
+      "%25, %26, %27, %28, %29, %30, %31}, [%33];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(a0), "r"(a1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait_tied(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+// acc[base .. base+15] += s * (32 loaded columns, as 16 pairs)
+__device__ __forceinline__ void promote16(float2 (&acc)[32], int base, const uint32_t (&r)[32],
+                                          float2 s) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    acc[base + c] = __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
+                               s, acc[base + c]);
+}
 
 struct KParams8 {
   const int* group_offsets;
@@ -86,7 +223,7 @@ struct KParams8 {
 };
 
 struct Tile8 {
-  int g, f0, nfeat, row0, nrows, k_blocks, row_tiles;
+  int g, f0, nfeat, row0, nrows, k_blocks, row_tiles;   // row0/nrows: the pair's rows
 };
 
 template <bool GATED>
@@ -101,7 +238,7 @@ __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* g
   ti.g = lo;
   const bool routed = lo < p.E;
   const int gbeg = go[lo], gend = go[lo + 1];
-  const int rt = (gend - gbeg + BMT - 1) / BMT;
+  const int rt = (gend - gbeg + PAIR_ROWS - 1) / PAIR_ROWS;
   const int local = t - ts[lo];
   const int f = local / rt;                    // feature tile outer, row tile inner
   const int r = local - f * rt;
@@ -109,8 +246,8 @@ __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* g
   const int feats = routed ? p.feat_routed : p.feat_shared;
   ti.f0 = f * fpt;
   ti.nfeat = min(fpt, feats - ti.f0);
-  ti.row0 = gbeg + r * BMT;
-  ti.nrows = min(BMT, gend - ti.row0);
+  ti.row0 = gbeg + r * PAIR_ROWS;
+  ti.nrows = min(PAIR_ROWS, gend - ti.row0);
   ti.k_blocks = routed ? p.kb_routed : p.kb_shared;
   ti.row_tiles = rt;
   return ti;
@@ -135,16 +272,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* b_smem = base + STAGES * A_BYTES;
   float* red = reinterpret_cast<float*>(base + DATA_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + DATA_BYTES + RED_BYTES);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* pfull = bars + 2 * STAGES;
-  uint64_t* pempty = pfull + 2;
+  uint64_t* full = bars;                 // even CTA: stage loaded in both CTAs (TMA bytes)
+  uint64_t* empty = bars + STAGES;       // stage consumed by the pair's MMAs
+  uint64_t* pfull = bars + 2 * STAGES;   // partial buffer written (both CTAs)
+  uint64_t* pempty = pfull + 2;          // even CTA: partial buffer read by all 16 epilogue warps
   uint64_t* teardown = pempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
   int* ts = reinterpret_cast<int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* go = p.group_offsets;
+  const uint32_t rank = cluster_rank();          // 0: issues the MMAs; 1: its peer
+  const int pair = (int)cluster_id_x();
+  const int npairs = (int)num_clusters_x();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -153,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&pfull[b]), 1);
-      mbar_init(smem_u32(&pempty[b]), kEpiWarps);
+      mbar_init(smem_u32(&pempty[b]), 2 * kEpiWarps);
     }
     mbar_init(smem_u32(teardown), 1);
     fence_mbarrier_init();
@@ -162,18 +302,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmWs);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 2) {
-    // tile prefix over groups: ceil(rows / 128) row tiles x feature tiles
+    // tile prefix over groups: ceil(rows / 256) row tiles x feature tiles
     int running = 0;
     for (int b0 = 0; b0 < p.G; b0 += 32) {
       const int g = b0 + lane;
       int cnt = 0;
       if (g < p.G) {
         const int rows = go[g + 1] - go[g];
-        cnt = (g < p.E ? p.ft_routed : p.ft_shared) * ((rows + BMT - 1) / BMT);
+        cnt = (g < p.E ? p.ft_routed : p.ft_shared) * ((rows + PAIR_ROWS - 1) / PAIR_ROWS);
       }
       int incl = cnt;
 #pragma unroll
@@ -188,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();        // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = ts[p.G];
@@ -205,14 +346,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const uint32_t full0 = map_to_rank(smem_u32(&full[0]), 0);   // the even CTA's barriers
+      for (int t = pair; t < total && ok; t += npairs) {
         const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
         const bool routed = ti.g < p.E;
         const CUtensorMap* wm = routed ? &tmW : &tmWs;
         const int wrow = (routed ? ti.g * p.rows_per_expert : 0) + ti.f0;
         const int up = routed ? p.up_routed : p.up_shared;
-        const int nb = GATED ? 2 : (ti.nfeat + 127) / 128;      // 128-row weight boxes
-        const uint32_t bytes = A_BYTES + nb * 128 * BK;
+        // gated: even CTA the gate rows, odd CTA the up rows; down: one 128-row half each
+        const int brow = GATED ? (rank == 0 ? wrow : wrow + up) : wrow + 128 * (int)rank;
+        const int arow = ti.row0 + BMT * (int)rank;
         const uint64_t pol_a = ti.row_tiles == 1 ? pol_last : pol_normal;
         const uint64_t pol_w = ti.row_tiles == 1 ? pol_first : pol_normal;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
@@ -221,41 +364,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(smem_u32(a_smem + stage * A_BYTES), &tmA, kb * BK, ti.row0, fb, pol_a);
-          const uint32_t b_dst = smem_u32(b_smem + stage * B_BYTES);
-          if (GATED) {
-            tma_load_2d(b_dst, wm, kb * BK, wrow, fb, pol_w);
-            tma_load_2d(b_dst + 128 * BK, wm, kb * BK, wrow + up, fb, pol_w);
-          } else {
-            for (int j = 0; j < nb; ++j)
-              tma_load_2d(b_dst + j * 128 * BK, wm, kb * BK, wrow + 128 * j, fb, pol_w);
-          }
+          // the even CTA expects both CTAs' bytes; the odd CTA's loads complete there
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (A_BYTES + B_BYTES));
+          const uint32_t fb = full0 + stage * (uint32_t)sizeof(uint64_t);
+          tma_load_2d_pair(smem_u32(a_smem + stage * A_BYTES), &tmA, kb * BK, arow, fb, pol_a);
+          tma_load_2d_pair(smem_u32(b_smem + stage * B_BYTES), wm, kb * BK, brow, fb, pol_w);
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      // no load may still be writing when the CTA leaves: wait until the MMAs
+      // have consumed the last load of every stage (which follows its arrival)
       for (int s = 0; s < STAGES; ++s)
         if ((issued >> s) & 1u)
-          mbar_wait_sleep(smem_u32(&full[s]), (parity >> s) & 1u, kTeardownLimitNs, p.status,
+          mbar_wait_sleep(smem_u32(&empty[s]), (parity >> s) & 1u, kTeardownLimitNs, p.status,
                           p.timeout_bit);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1 && lane == 0 && rank == 0) {
       // ----------------------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       uint32_t kcount = 0;          // K blocks issued so far: partial buffer = kcount & 1
       bool ok = true, any = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = pair; t < total && ok; t += npairs) {
         const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
-        const int n = GATED ? 256 : ((ti.nfeat + 127) / 128) * 128;
-        const uint32_t idesc = idesc_e4m3_m128(n);
         for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
           const uint32_t pb = kcount & 1u;
           const uint32_t use = kcount >> 1;
-          if (!mbar_wait_sleep(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns, p.status,
-                               p.timeout_bit) ||
+          if (!mbar_wait_sleep(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns,
+                               p.status, p.timeout_bit) ||
               !mbar_wait_sleep(smem_u32(&full[stage]), phase, p.wait_limit_ns, p.status,
                                p.timeout_bit)) {
             ok = false;
@@ -267,38 +404,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b_desc = smem_desc_sw128(smem_u32(b_smem + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)   // +32 bytes per K step = 2 in the address field
-            umma_e4m3(d0, a_desc + 2 * kk, b_desc + 2 * kk, idesc, kk != 0);
-          umma_commit(smem_u32(&empty[stage]));
-          umma_commit(smem_u32(&pfull[pb]));
+            umma_e4m3_pair(d0, a_desc + 2 * kk, b_desc + 2 * kk, kIdescPair, kk != 0);
+          umma_commit_both(smem_u32(&empty[stage]));
+          umma_commit_both(smem_u32(&pfull[pb]));
           any = true;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (any) {
-        umma_commit(smem_u32(teardown));
+        umma_commit_both(smem_u32(teardown));
         mbar_wait_sleep(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
       }
+    } else if (warp == 1 && lane == 0) {
+      // odd CTA: wait for the pair's last MMAs before tensor memory is freed
+      bool any = false;
+      for (int t = pair; t < total; t += npairs) any = true;
+      if (any) mbar_wait_sleep(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
     }
     __syncwarp();
   } else {
     regs_inc<kEpilogueRegs>();
     // ------------------------------------------------- promotion and epilogue
-    // Thread = one activation row of the tile (its TMEM lane) and one half of
-    // the tile's columns.  Every epilogue warp walks the same tiles and K
-    // blocks and, for gated tiles, passes one named barrier per tile whatever
-    // happens: after an expired wait it keeps walking without further waits,
-    // loads or stores.
+    // Thread = one activation row of this CTA's half of the tile (its TMEM
+    // lane) and one half of the tile's columns.  Every epilogue warp walks the
+    // same tiles and K blocks and, for gated tiles, passes one named barrier
+    // per tile whatever happens: after an expired wait it keeps walking
+    // without further waits, loads or stores.  Rows past the group's end are
+    // computed by the MMA but neither promoted nor stored.
     const int ew = warp - 4;              // 0..7
     const int q = warp & 3;               // TMEM lane quadrant
     const int hh = ew >> 2;               // column half
-    const int r = q * 32 + lane;          // row within the tile
+    const int r = q * 32 + lane;          // row within this CTA's 128
+    const uint32_t pempty0 = map_to_rank(smem_u32(&pempty[0]), 0);
+    const uint32_t pempty1 = map_to_rank(smem_u32(&pempty[1]), 0);
     uint32_t kcount = 0;
     int tiles_done = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tiles_done) {
+    for (int t = pair; t < total; t += npairs, ++tiles_done) {
       const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
       const bool routed = ti.g < p.E;
-      const bool live = r < ti.nrows;
+      const int my_row0 = ti.row0 + BMT * (int)rank;
+      const int my_rows = max(0, min(BMT, ti.nrows - BMT * (int)rank));
+      const bool live = r < my_rows;
+      const bool warp_live = q * 32 < my_rows;
       const bool any_cols = GATED || hh * 128 < ti.nfeat;
       const int sw_kb = ti.k_blocks;
       const float* sw = routed ? p.sw_routed + (size_t)ti.g * (p.rows_per_expert / 128) * sw_kb
@@ -307,10 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int up = routed ? p.up_routed : p.up_shared;
       const float* swa = sw + (size_t)((ti.f0 + (GATED ? 0 : hh * 128)) / 128) * sw_kb;
       const float* swb = sw + (size_t)((up + ti.f0) / 128) * sw_kb;
-      const float* sa_row = p.sa + (size_t)(ti.row0 + r) * p.sa_ld;
-      float nxt_a = live ? sa_row[0] : 0.f;
-      float nxt_wa = swa[0];
-      float nxt_wb = GATED ? swb[0] : 0.f;
+      // rows past the group read the pair's first row instead (in bounds, unused)
+      const float* sa_row = p.sa + (size_t)(live ? my_row0 + r : ti.row0) * p.sa_ld;
+      float nxt_a = ldg_ahead(sa_row);
+      float nxt_wa = ldg_ahead(swa);
+      float nxt_wb = GATED ? ldg_ahead(swb) : 0.f;
 
       // gated: g and u of 64 features; down: 128 features.  Pairs of columns
       // are updated by one packed fp32 FMA (same rounding as two scalar FMAs).
@@ -323,61 +472,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u;
         const uint32_t use = kcount >> 1;
-        const float sa_cur = nxt_a;
+        const float sa_cur = live ? nxt_a : 0.f;
         const float s_a = nxt_wa * sa_cur;
         const float s_b = (GATED ? nxt_wb : nxt_wa) * sa_cur;
         if (kb + 1 < ti.k_blocks) {                   // next block's factors, fetched early
-          nxt_a = live ? sa_row[kb + 1] : 0.f;
-          nxt_wa = swa[kb + 1];
-          if (GATED) nxt_wb = swb[kb + 1];
+          nxt_a = ldg_ahead(sa_row + kb + 1);
+          nxt_wa = ldg_ahead(swa + kb + 1);
+          if (GATED) nxt_wb = ldg_ahead(swb + kb + 1);
         }
         if (ok)
           ok = mbar_wait_sleep_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns, p.status,
                                     p.timeout_bit);
         if (!ok) continue;
         tc_fence_after();
-        // the partial buffer goes back to the MMA as soon as it has been read
+        // the partial buffer goes back to the MMA issuer as soon as it has been read
         auto release = [&]() {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&pempty[pb]));
-        };
-        if (any_cols) {
-          const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride;
-          float v[64];
-          const float2 sa2 = make_float2(s_a, s_a), sb2 = make_float2(s_b, s_b);
-          if (GATED) {
-            // gate columns hh*64 .. +63 and up columns 128 + hh*64 .. +63
-            const uint32_t g0 = tl + hh * 64, u0 = tl + 128 + hh * 64;
-            tmem_ld_16x4(g0, g0 + 16, u0, u0 + 16, v);
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              acc_a[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[c]);
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              acc_b[c] = __ffma2_rn(make_float2(v[32 + 2 * c], v[33 + 2 * c]), sb2, acc_b[c]);
-            tmem_ld_16x4(g0 + 32, g0 + 48, u0 + 32, u0 + 48, v);
-            release();
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              acc_a[16 + c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[16 + c]);
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              acc_b[16 + c] =
-                  __ffma2_rn(make_float2(v[32 + 2 * c], v[33 + 2 * c]), sb2, acc_b[16 + c]);
-          } else {
-            // columns hh*128 .. +127, one weight scale block
-            const uint32_t c0 = tl + hh * 128;
-            tmem_ld_16x4(c0, c0 + 16, c0 + 32, c0 + 48, v);
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              acc_a[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_a[c]);
-            tmem_ld_16x4(c0 + 64, c0 + 80, c0 + 96, c0 + 112, v);
-            release();
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              acc_b[c] = __ffma2_rn(make_float2(v[2 * c], v[2 * c + 1]), sa2, acc_b[c]);
+          if (lane == 0) {
+            if (rank == 0) mbar_arrive(smem_u32(&pempty[pb]));
+            else mbar_arrive_remote_signal(pb ? pempty1 : pempty0);
           }
+        };
+        if (any_cols && warp_live) {
+          const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride;
+          const float2 sa2 = make_float2(s_a, s_a), sb2 = make_float2(s_b, s_b);
+          uint32_t ra[32], rb[32];
+          // gated: gate columns hh*64 .. +63 -> acc_a, up columns 128 + hh*64 .. -> acc_b;
+          // down: columns hh*128 .. +63 -> acc_a, +64 .. +127 -> acc_b (one scale block).
+          const uint32_t c0 = GATED ? tl + hh * 64 : tl + hh * 128;
+          const uint32_t c1 = GATED ? tl + 128 + hh * 64 : tl + hh * 128 + 64;
+          tmem_ld_2x16(c0, c0 + 16, ra);
+          tmem_ld_wait_tied(ra);
+          tmem_ld_2x16(c1, c1 + 16, rb);
+          promote16(acc_a, 0, ra, sa2);
+          tmem_ld_wait_tied(rb);
+          tmem_ld_2x16(c0 + 32, c0 + 48, ra);
+          promote16(acc_b, 0, rb, sb2);
+          tmem_ld_wait_tied(ra);
+          tmem_ld_2x16(c1 + 32, c1 + 48, rb);
+          promote16(acc_a, 16, ra, sa2);
+          tmem_ld_wait_tied(rb);
+          release();
+          promote16(acc_b, 16, rb, sb2);
         } else {
           release();
         }
@@ -401,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && live) {
           const float m = fmaxf(red_p[r * 2], red_p[r * 2 + 1]);
           const float s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-          const int row = ti.row0 + r;
+          const int row = my_row0 + r;
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + (size_t)row * p.ldd +
                                                 ti.f0 + hh * 64);
 #pragma unroll
@@ -419,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (hh == 0) p.sd[(size_t)row * (p.ldd / 128) + ti.f0 / 128] = s;
         }
       } else if (ok && live && any_cols) {
-        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(ti.row0 + r) * p.ldd +
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(my_row0 + r) * p.ldd +
                            ti.f0 + hh * 128;
         uint4* dst = reinterpret_cast<uint4*>(y);
 #pragma unroll
@@ -438,11 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // Neither CTA leaves (or frees tensor memory) while the other may still
+  // arrive on its barriers or have the tensor core read its shared memory.
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -483,6 +623,47 @@ cudaError_t check_register_split() {
   cudaError_t e = cudaFuncGetAttributes(&attr, grouped_gemm_fp8_kernel<GATED>);
   if (e != cudaSuccess) return e;
   return attr.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+cudaLaunchConfig_t pair_config(int pairs, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// CTA pairs that can be resident at once, per device (a persistent grid of
+// more pairs would leave some waiting for others to finish).
+constexpr int kMaxDevices = 64;
+int g_pairs[kMaxDevices][2];
+std::mutex g_pairs_mu;
+
+template <bool GATED>
+cudaError_t resident_pairs(int num_sms, int* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_pairs_mu);
+  if (g_pairs[dev][GATED] == 0) {
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(num_sms / 2, nullptr, attr);
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_fp8_kernel<GATED>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    g_pairs[dev][GATED] = min(clusters, num_sms / 2);
+  }
+  *out = g_pairs[dev][GATED];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -535,12 +716,15 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   p.status = a.status;
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
-  if (a.gated) {
-    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
-  } else {
-    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
-  }
-  return cudaGetLastError();
+
+  int pairs = 0;
+  cudaError_t e = a.gated ? resident_pairs<true>(a.num_ctas, &pairs)
+                          : resident_pairs<false>(a.num_ctas, &pairs);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = pair_config(pairs, st, attr);
+  if (a.gated) return cudaLaunchKernelEx(&cfg, grouped_gemm_fp8_kernel<true>, tmA, tmW, tmWs, p);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_fp8_kernel<false>, tmA, tmW, tmWs, p);
 }
 
 }  // namespace moe
