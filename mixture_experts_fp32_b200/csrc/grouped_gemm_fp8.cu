@@ -14,51 +14,45 @@
 // fp32 register accumulators with its scale ("promotion").  Two partial
 // buffers let the tensor core run one K block ahead of the promotion.
 //
-// CTA pairs.  A tile is 256 activation rows x 256 weight rows, computed by the
-// two CTAs of a cluster with cta_group::2 MMAs (M = 256, N = 256): each CTA
-// stages its own 128 activation rows and one half (128 rows) of the weight
-// tile, and receives its 128 rows x all 256 columns in its own tensor memory.
-// Per 128-K block a CTA moves 32 KB through shared memory instead of the 48 KB
-// of a one-CTA 128 x 256 tile, and shared-memory bandwidth (TMA writes plus
-// tensor-core operand reads) is what bounds a one-CTA e4m3 tile on sm_100.
-// The even CTA of the pair issues the MMAs and owns the stage barriers: both
-// CTAs' TMA loads complete their bytes on it (cta_group::2 form of the load),
-// and the odd CTA's epilogue warps return partial buffers to it by remote
-// mbarrier arrivals.  No load is multicast.
+// One CTA per tile of 128 activation rows x 256 weight rows (M = 128, N = 256).
+// What bounds this loop is the hand-off of the two partial buffers: with a new
+// scale every 128 K, tensor memory (512 columns) holds two K blocks of partials,
+// and an MMA into a buffer must wait until the promotion has read it.  Tiles
+// of 256 rows on CTA pairs (cta_group::2, half the weight tile staged per CTA)
+// move less shared memory per K block but hit the same hand-off bound and pad
+// groups to 256 rows; measured on the 8192-token, 256-expert prefill they were
+// slower than this one-CTA form.
 //
 // Rows of activations take the MMA's M side and weight rows its N side: a TMEM
 // lane is one activation row, so the activation scale of a K block is one
 // register per thread and the weight scale one per 128 columns; promotion is
 // one FMA per value, and each thread writes its row contiguously.
 //
-//   gated: a pair tile owns 128 features of h: the even CTA stages their 128
-//          gate rows, the odd CTA their 128 up rows (N = 256), so g and u of a
-//          feature sit in the same TMEM lane of both CTAs.  After the last K
-//          block h = silu(g) * u is quantised per 1x128 group (the tile's 128
-//          features are one group) into e4m3 codes and an fp32 scale.
-//   down:  a pair tile owns 256 output features (two weight scale blocks, one
-//          staged by each CTA); y is written in bf16.
+//   gated: a tile owns 128 features of h: the B operand stacks the matching
+//          128 gate rows and 128 up rows (N = 256), so g and u of a feature sit
+//          in the same TMEM lane.  After the last K block h = silu(g) * u is
+//          quantised per 1x128 group (the tile's 128 features are one group)
+//          into e4m3 codes and an fp32 scale.
+//   down:  a tile owns up to 256 output features (two weight scale blocks); y
+//          is written in bf16.
 //
 // Three warpgroups (384 threads).  Warpgroup 0: warp 0 issues TMA loads, warp 1
-// owns tensor memory and, in the even CTA, issues the MMAs; it gives registers
-// back (setmaxnreg.dec).  Warpgroups 1 and 2
-// (8 warps) promote and finish, with the registers warpgroup 0 released: warp w
-// reads TMEM lanes 32*(w%4)... and one half of the tile's columns, 128 fp32
-// accumulators a thread.  Every wait is bounded and suspends rather than spins.
+// owns tensor memory and issues the MMAs; it gives registers back
+// (setmaxnreg.dec).  Warpgroups 1 and 2 (8 warps) promote and finish, with the
+// registers warpgroup 0 released: warp w reads TMEM lanes 32*(w%4)... and one
+// half of the tile's columns, 128 fp32 accumulators a thread.  Every wait is
+// bounded and suspends rather than spins.
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
-
-#include <mutex>
 
 #include "moe_internal.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int BMT = 128;           // activation rows per CTA (a pair covers 2 * BMT)
-constexpr int PAIR_ROWS = 2 * BMT;
+constexpr int BMT = 128;           // activation rows per tile (MMA M)
 constexpr int BK = 128;            // e4m3 elements (= bytes) per K block: one scale group
-constexpr int BNW = 256;           // weight rows per pair tile (MMA N); 128 staged per CTA
+constexpr int BNW = 256;           // weight rows per tile (MMA N)
 constexpr int kEpiWarps = 8;       // two per TMEM lane quadrant, each half of the columns
 constexpr int kThreads = 384;
 // 12 warps leave each SM sub-partition three warps: 168 registers a thread at
@@ -72,91 +66,14 @@ static_assert(128 * kProducerRegs + 256 * kEpilogueRegs == kThreads * kLaunchReg
               "register shares must add up to the launch's registers");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPartStride = 256;   // TMEM columns between the two partial buffers
-constexpr int A_BYTES = BMT * BK;              // 16 KB: this CTA's activation rows
-constexpr int B_BYTES = (BNW / 2) * BK;        // 16 KB: this CTA's half of the weight rows
-constexpr int STAGES = 6;
+constexpr int A_BYTES = BMT * BK;              // 16 KB: the tile's activation rows
+constexpr int B_BYTES = BNW * BK;              // 32 KB: all 256 weight rows
+constexpr int STAGES = 4;
 constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
 constexpr int RED_BYTES = 2 * BMT * 2 * 4;    // h amax halves [tile parity][row][half]
-constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 2048;
+constexpr int kGroupSlots = kMaxExperts + 4;   // >= groups + 1
+constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 256 + 2 * 4 * kGroupSlots;
 constexpr unsigned long long kTeardownLimitNs = 1000000000ull;
-
-// ------------------------------------------------------- CTA-pair primitives
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_id_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t num_clusters_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
-// Address of the same shared-memory object in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
-  return r;
-}
-// Remote arrival that publishes no memory: returning a tensor-memory partial
-// buffer, whose reads tcgen05.wait::ld has already completed and
-// tcgen05.fence::before_thread_sync has ordered before this arrival.  A
-// cluster-scope release here would cost a cluster-wide fence on the MMA's
-// critical path.
-__device__ __forceinline__ void mbar_arrive_remote_signal(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// 2-D tiled TMA load (no multicast) into this CTA's shared memory whose bytes
-// complete on an mbarrier of either CTA of the pair (here: the even CTA's).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, int x, int y,
-                                                 uint32_t bar_cluster, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cluster), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256.
-__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrive on the mbarrier at this shared-memory offset in both CTAs of the pair
-// once the pair MMAs this thread issued so far have completed.
-__device__ __forceinline__ void umma_commit_both(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar), "h"((uint16_t)0x3)
-      : "memory");
-}
-// kind::f8f6f4 instruction descriptor for M = 256, N = 256, e4m3 x e4m3 -> f32.
-constexpr uint32_t kIdescPair = (1u << 4) | ((uint32_t)(BNW >> 3) << 17) |
-                                ((uint32_t)(PAIR_ROWS >> 4) << 24);
 
 // A scale fetched ahead of its use: the asm keeps the load where it is written
 // (the compiler may not sink it next to the use and expose its latency).
@@ -223,7 +140,7 @@ struct KParams8 {
 };
 
 struct Tile8 {
-  int g, f0, nfeat, row0, nrows, k_blocks, row_tiles;   // row0/nrows: the pair's rows
+  int g, f0, nfeat, row0, nrows, k_blocks, row_tiles;
 };
 
 template <bool GATED>
@@ -238,7 +155,7 @@ __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* g
   ti.g = lo;
   const bool routed = lo < p.E;
   const int gbeg = go[lo], gend = go[lo + 1];
-  const int rt = (gend - gbeg + PAIR_ROWS - 1) / PAIR_ROWS;
+  const int rt = (gend - gbeg + BMT - 1) / BMT;
   const int local = t - ts[lo];
   const int f = local / rt;                    // feature tile outer, row tile inner
   const int r = local - f * rt;
@@ -246,8 +163,8 @@ __device__ __forceinline__ Tile8 decode_tile8(int t, const int* ts, const int* g
   const int feats = routed ? p.feat_routed : p.feat_shared;
   ti.f0 = f * fpt;
   ti.nfeat = min(fpt, feats - ti.f0);
-  ti.row0 = gbeg + r * PAIR_ROWS;
-  ti.nrows = min(PAIR_ROWS, gend - ti.row0);
+  ti.row0 = gbeg + r * BMT;
+  ti.nrows = min(BMT, gend - ti.row0);
   ti.k_blocks = routed ? p.kb_routed : p.kb_shared;
   ti.row_tiles = rt;
   return ti;
@@ -272,19 +189,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* b_smem = base + STAGES * A_BYTES;
   float* red = reinterpret_cast<float*>(base + DATA_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + DATA_BYTES + RED_BYTES);
-  uint64_t* full = bars;                 // even CTA: stage loaded in both CTAs (TMA bytes)
-  uint64_t* empty = bars + STAGES;       // stage consumed by the pair's MMAs
-  uint64_t* pfull = bars + 2 * STAGES;   // partial buffer written (both CTAs)
-  uint64_t* pempty = pfull + 2;          // even CTA: partial buffer read by all 16 epilogue warps
+  uint64_t* full = bars;                 // stage loaded (TMA bytes)
+  uint64_t* empty = bars + STAGES;       // stage consumed by the MMAs
+  uint64_t* pfull = bars + 2 * STAGES;   // partial buffer written
+  uint64_t* pempty = pfull + 2;          // partial buffer read by all epilogue warps
   uint64_t* teardown = pempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(teardown + 1);
-  int* ts = reinterpret_cast<int*>(tmem_holder + 1);
+  int* ts = reinterpret_cast<int*>(tmem_holder + 1);   // first tile of each group
+  int* gos = ts + kGroupSlots;                            // group row offsets, staged
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int* go = p.group_offsets;
-  const uint32_t rank = cluster_rank();          // 0: issues the MMAs; 1: its peer
-  const int pair = (int)cluster_id_x();
-  const int npairs = (int)num_clusters_x();
+  const int* go = gos;
+  const int cta = blockIdx.x, nctas = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -293,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&pfull[b]), 1);
-      mbar_init(smem_u32(&pempty[b]), 2 * kEpiWarps);
+      mbar_init(smem_u32(&pempty[b]), kEpiWarps);
     }
     mbar_init(smem_u32(teardown), 1);
     fence_mbarrier_init();
@@ -302,18 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmWs);
   }
   if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish_pair();
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
   }
   if (warp == 2) {
-    // tile prefix over groups: ceil(rows / 256) row tiles x feature tiles
+    // tile prefix over groups: ceil(rows / 128) row tiles x feature tiles
     int running = 0;
     for (int b0 = 0; b0 < p.G; b0 += 32) {
       const int g = b0 + lane;
       int cnt = 0;
       if (g < p.G) {
-        const int rows = go[g + 1] - go[g];
-        cnt = (g < p.E ? p.ft_routed : p.ft_shared) * ((rows + PAIR_ROWS - 1) / PAIR_ROWS);
+        const int beg = p.group_offsets[g], end = p.group_offsets[g + 1];
+        gos[g] = beg;
+        const int rows = end - beg;
+        cnt = (g < p.E ? p.ft_routed : p.ft_shared) * ((rows + BMT - 1) / BMT);
       }
       int incl = cnt;
 #pragma unroll
@@ -324,11 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < p.G) ts[g] = running + incl - cnt;
       running += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) ts[p.G] = running;
+    if (lane == 0) {
+      ts[p.G] = running;
+      gos[p.G] = p.group_offsets[p.G];
+    }
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();        // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = ts[p.G];
@@ -346,16 +266,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
       bool ok = true;
-      const uint32_t full0 = map_to_rank(smem_u32(&full[0]), 0);   // the even CTA's barriers
-      for (int t = pair; t < total && ok; t += npairs) {
+      for (int t = cta; t < total && ok; t += nctas) {
         const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
         const bool routed = ti.g < p.E;
         const CUtensorMap* wm = routed ? &tmW : &tmWs;
         const int wrow = (routed ? ti.g * p.rows_per_expert : 0) + ti.f0;
         const int up = routed ? p.up_routed : p.up_shared;
-        // gated: even CTA the gate rows, odd CTA the up rows; down: one 128-row half each
-        const int brow = GATED ? (rank == 0 ? wrow : wrow + up) : wrow + 128 * (int)rank;
-        const int arow = ti.row0 + BMT * (int)rank;
+        const int brow0 = wrow, brow1 = GATED ? wrow + up : wrow + 128;
+        const int arow = ti.row0;
         const uint64_t pol_a = ti.row_tiles == 1 ? pol_last : pol_normal;
         const uint64_t pol_w = ti.row_tiles == 1 ? pol_first : pol_normal;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
@@ -364,11 +282,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // the even CTA expects both CTAs' bytes; the odd CTA's loads complete there
-          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (A_BYTES + B_BYTES));
-          const uint32_t fb = full0 + stage * (uint32_t)sizeof(uint64_t);
-          tma_load_2d_pair(smem_u32(a_smem + stage * A_BYTES), &tmA, kb * BK, arow, fb, pol_a);
-          tma_load_2d_pair(smem_u32(b_smem + stage * B_BYTES), wm, kb * BK, brow, fb, pol_w);
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+          tma_load_2d(smem_u32(a_smem + stage * A_BYTES), &tmA, kb * BK, arow, fb, pol_a);
+          tma_load_2d(smem_u32(b_smem + stage * B_BYTES), wm, kb * BK, brow0, fb, pol_w);
+          tma_load_2d(smem_u32(b_smem + stage * B_BYTES + 128 * BK), wm, kb * BK, brow1, fb, pol_w);
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -380,15 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((issued >> s) & 1u)
           mbar_wait_sleep(smem_u32(&empty[s]), (parity >> s) & 1u, kTeardownLimitNs, p.status,
                           p.timeout_bit);
-    } else if (warp == 1 && lane == 0 && rank == 0) {
+    } else if (warp == 1 && lane == 0) {
       // ----------------------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       uint32_t kcount = 0;          // K blocks issued so far: partial buffer = kcount & 1
       bool ok = true, any = false;
-      for (int t = pair; t < total && ok; t += npairs) {
-        const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
-        for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
+      for (int t = cta; t < total && ok; t += nctas) {
+        const int k_blocks = decode_tile8<GATED>(t, ts, go, p).k_blocks;
+        for (int kb = 0; kb < k_blocks; ++kb, ++kcount) {
           const uint32_t pb = kcount & 1u;
           const uint32_t use = kcount >> 1;
           if (!mbar_wait_sleep(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns,
@@ -404,29 +322,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b_desc = smem_desc_sw128(smem_u32(b_smem + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)   // +32 bytes per K step = 2 in the address field
-            umma_e4m3_pair(d0, a_desc + 2 * kk, b_desc + 2 * kk, kIdescPair, kk != 0);
-          umma_commit_both(smem_u32(&empty[stage]));
-          umma_commit_both(smem_u32(&pfull[pb]));
+            umma_e4m3(d0, a_desc + 2 * kk, b_desc + 2 * kk, idesc_e4m3_m128(BNW), kk != 0);
+          umma_commit(smem_u32(&empty[stage]));
+          umma_commit(smem_u32(&pfull[pb]));
           any = true;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (any) {
-        umma_commit_both(smem_u32(teardown));
+        umma_commit(smem_u32(teardown));
         mbar_wait_sleep(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
       }
-    } else if (warp == 1 && lane == 0) {
-      // odd CTA: wait for the pair's last MMAs before tensor memory is freed
-      bool any = false;
-      for (int t = pair; t < total; t += npairs) any = true;
-      if (any) mbar_wait_sleep(smem_u32(teardown), 0, kTeardownLimitNs, p.status, p.timeout_bit);
     }
     __syncwarp();
   } else {
     regs_inc<kEpilogueRegs>();
     // ------------------------------------------------- promotion and epilogue
-    // Thread = one activation row of this CTA's half of the tile (its TMEM
-    // lane) and one half of the tile's columns.  Every epilogue warp walks the
+    // Thread = one activation row of the tile (its TMEM lane) and one half of
+    // the tile's columns.  Every epilogue warp walks the
     // same tiles and K blocks and, for gated tiles, passes one named barrier
     // per tile whatever happens: after an expired wait it keeps walking
     // without further waits, loads or stores.  Rows past the group's end are
@@ -435,31 +348,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;               // TMEM lane quadrant
     const int hh = ew >> 2;               // column half
     const int r = q * 32 + lane;          // row within this CTA's 128
-    const uint32_t pempty0 = map_to_rank(smem_u32(&pempty[0]), 0);
-    const uint32_t pempty1 = map_to_rank(smem_u32(&pempty[1]), 0);
-    uint32_t kcount = 0;
-    int tiles_done = 0;
-    bool ok = true;
-    for (int t = pair; t < total; t += npairs, ++tiles_done) {
+    // Per-tile state of this thread; the next tile's is set up (and its first
+    // scales requested) before the current tile's finishing work, so that the
+    // loads' latency hides behind it.
+    struct EpiTile {
+      int row0, rows, f0, nfeat, k_blocks;
+      const float* sa_row;
+      const float* swa;
+      const float* swb;
+    };
+    auto setup = [&](int t, EpiTile& e, float& a0, float& wa0, float& wb0) {
       const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
       const bool routed = ti.g < p.E;
-      const int my_row0 = ti.row0 + BMT * (int)rank;
-      const int my_rows = max(0, min(BMT, ti.nrows - BMT * (int)rank));
-      const bool live = r < my_rows;
-      const bool warp_live = q * 32 < my_rows;
-      const bool any_cols = GATED || hh * 128 < ti.nfeat;
-      const int sw_kb = ti.k_blocks;
-      const float* sw = routed ? p.sw_routed + (size_t)ti.g * (p.rows_per_expert / 128) * sw_kb
+      e.row0 = ti.row0;
+      e.rows = ti.nrows;
+      e.f0 = ti.f0;
+      e.nfeat = ti.nfeat;
+      e.k_blocks = ti.k_blocks;
+      const float* sw = routed ? p.sw_routed + (size_t)ti.g * (p.rows_per_expert / 128) * ti.k_blocks
                                : p.sw_shared;
       // weight scale rows: gated -> gate block and up block of f0; down -> block of this half
       const int up = routed ? p.up_routed : p.up_shared;
-      const float* swa = sw + (size_t)((ti.f0 + (GATED ? 0 : hh * 128)) / 128) * sw_kb;
-      const float* swb = sw + (size_t)((up + ti.f0) / 128) * sw_kb;
-      // rows past the group read the pair's first row instead (in bounds, unused)
-      const float* sa_row = p.sa + (size_t)(live ? my_row0 + r : ti.row0) * p.sa_ld;
-      float nxt_a = ldg_ahead(sa_row);
-      float nxt_wa = ldg_ahead(swa);
-      float nxt_wb = GATED ? ldg_ahead(swb) : 0.f;
+      e.swa = sw + (size_t)((ti.f0 + (GATED ? 0 : hh * 128)) / 128) * ti.k_blocks;
+      e.swb = sw + (size_t)((up + ti.f0) / 128) * ti.k_blocks;
+      // rows past the group read the tile's first row instead (in bounds, unused)
+      e.sa_row = p.sa + (size_t)(r < e.rows ? e.row0 + r : ti.row0) * p.sa_ld;
+      a0 = ldg_ahead(e.sa_row);
+      wa0 = ldg_ahead(e.swa);
+      wb0 = GATED ? ldg_ahead(e.swb) : 0.f;
+    };
+    uint32_t kcount = 0;
+    int tiles_done = 0;
+    bool ok = true;
+    EpiTile cur;
+    float nxt_a = 0.f, nxt_wa = 0.f, nxt_wb = 0.f;
+    if (cta < total) setup(cta, cur, nxt_a, nxt_wa, nxt_wb);
+    for (int t = cta; t < total; t += nctas, ++tiles_done) {
+      const bool live = r < cur.rows;
+      const bool warp_live = q * 32 < cur.rows;
+      const bool any_cols = GATED || hh * 128 < cur.nfeat;
 
       // gated: g and u of 64 features; down: 128 features.  Pairs of columns
       // are updated by one packed fp32 FMA (same rounding as two scalar FMAs).
@@ -469,16 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_a[c] = make_float2(0.f, 0.f);
         acc_b[c] = make_float2(0.f, 0.f);
       }
-      for (int kb = 0; kb < ti.k_blocks; ++kb, ++kcount) {
+      for (int kb = 0; kb < cur.k_blocks; ++kb, ++kcount) {
         const uint32_t pb = kcount & 1u;
         const uint32_t use = kcount >> 1;
         const float sa_cur = live ? nxt_a : 0.f;
         const float s_a = nxt_wa * sa_cur;
         const float s_b = (GATED ? nxt_wb : nxt_wa) * sa_cur;
-        if (kb + 1 < ti.k_blocks) {                   // next block's factors, fetched early
-          nxt_a = ldg_ahead(sa_row + kb + 1);
-          nxt_wa = ldg_ahead(swa + kb + 1);
-          if (GATED) nxt_wb = ldg_ahead(swb + kb + 1);
+        if (kb + 1 < cur.k_blocks) {                  // next block's factors, fetched early
+          nxt_a = ldg_ahead(cur.sa_row + kb + 1);
+          nxt_wa = ldg_ahead(cur.swa + kb + 1);
+          if (GATED) nxt_wb = ldg_ahead(cur.swb + kb + 1);
         }
         if (ok)
           ok = mbar_wait_sleep_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns, p.status,
@@ -489,10 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto release = [&]() {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            if (rank == 0) mbar_arrive(smem_u32(&pempty[pb]));
-            else mbar_arrive_remote_signal(pb ? pempty1 : pempty0);
-          }
+          if (lane == 0) mbar_arrive(smem_u32(&pempty[pb]));
         };
         if (any_cols && warp_live) {
           const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + pb * kPartStride;
@@ -520,16 +444,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
+      const EpiTile fin = cur;                       // the tile being finished
+      if (t + nctas < total) setup(t + nctas, cur, nxt_a, nxt_wa, nxt_wb);
+
       if (GATED) {
         // h = silu(g) * u over this thread's 64 features; the row's scale needs
-        // the max over both halves (the partner warp holds the other 64)
+        // the max over both halves (the partner warp holds the other 64).
+        // silu's quotient uses the fast reciprocal division (about 2 ulp; its
+        // denominator 1 + e^-g is >= 1 and saturates to +inf, giving -0 for
+        // g -> -inf): h is quantised to 3 mantissa bits right after.
         float amax = 0.f;
         float hv[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float g = (c & 1) ? acc_a[c >> 1].y : acc_a[c >> 1].x;
           const float u = (c & 1) ? acc_b[c >> 1].y : acc_b[c >> 1].x;
-          hv[c] = g / (1.0f + __expf(-g)) * u;
+          hv[c] = __fdividef(g, 1.0f + __expf(-g)) * u;
           amax = fmaxf(amax, fabsf(hv[c]));
         }
         float* red_p = red + (tiles_done & 1) * BMT * 2;
@@ -538,9 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && live) {
           const float m = fmaxf(red_p[r * 2], red_p[r * 2 + 1]);
           const float s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
-          const int row = my_row0 + r;
+          // codes: h * (1/s) rounded to e4m3, the reciprocal once per row
+          const float inv = __frcp_rn(s);
+          const int row = fin.row0 + r;
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.d) + (size_t)row * p.ldd +
-                                                ti.f0 + hh * 64);
+                                                fin.f0 + hh * 64);
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
             uint4 o;
@@ -548,16 +480,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int c = w4 * 16 + j * 4;
-              ow[j] = e4m3x4(__fdiv_rn(hv[c], s), __fdiv_rn(hv[c + 1], s),
-                             __fdiv_rn(hv[c + 2], s), __fdiv_rn(hv[c + 3], s));
+              ow[j] = e4m3x4(hv[c] * inv, hv[c + 1] * inv, hv[c + 2] * inv, hv[c + 3] * inv);
             }
             dst[w4] = o;
           }
-          if (hh == 0) p.sd[(size_t)row * (p.ldd / 128) + ti.f0 / 128] = s;
+          if (hh == 0) p.sd[(size_t)row * (p.ldd / 128) + fin.f0 / 128] = s;
         }
       } else if (ok && live && any_cols) {
-        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(my_row0 + r) * p.ldd +
-                           ti.f0 + hh * 128;
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(fin.row0 + r) * p.ldd +
+                           fin.f0 + hh * 128;
         uint4* dst = reinterpret_cast<uint4*>(y);
 #pragma unroll
         for (int w8 = 0; w8 < 16; ++w8) {
@@ -575,14 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // Neither CTA leaves (or frees tensor memory) while the other may still
-  // arrive on its barriers or have the tensor core read its shared memory.
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -623,47 +551,6 @@ cudaError_t check_register_split() {
   cudaError_t e = cudaFuncGetAttributes(&attr, grouped_gemm_fp8_kernel<GATED>);
   if (e != cudaSuccess) return e;
   return attr.numRegs == kLaunchRegs ? cudaSuccess : cudaErrorInvalidConfiguration;
-}
-
-cudaLaunchConfig_t pair_config(int pairs, cudaStream_t st, cudaLaunchAttribute* attr) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = st;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cfg;
-}
-
-// CTA pairs that can be resident at once, per device (a persistent grid of
-// more pairs would leave some waiting for others to finish).
-constexpr int kMaxDevices = 64;
-int g_pairs[kMaxDevices][2];
-std::mutex g_pairs_mu;
-
-template <bool GATED>
-cudaError_t resident_pairs(int num_sms, int* out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_pairs_mu);
-  if (g_pairs[dev][GATED] == 0) {
-    cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = pair_config(num_sms / 2, nullptr, attr);
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_fp8_kernel<GATED>, &cfg);
-    if (e != cudaSuccess) return e;
-    if (clusters < 1) return cudaErrorInvalidConfiguration;
-    g_pairs[dev][GATED] = min(clusters, num_sms / 2);
-  }
-  *out = g_pairs[dev][GATED];
-  return cudaSuccess;
 }
 
 }  // namespace
@@ -717,14 +604,11 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
 
-  int pairs = 0;
-  cudaError_t e = a.gated ? resident_pairs<true>(a.num_ctas, &pairs)
-                          : resident_pairs<false>(a.num_ctas, &pairs);
-  if (e != cudaSuccess) return e;
-  cudaLaunchAttribute attr[1];
-  const cudaLaunchConfig_t cfg = pair_config(pairs, st, attr);
-  if (a.gated) return cudaLaunchKernelEx(&cfg, grouped_gemm_fp8_kernel<true>, tmA, tmW, tmWs, p);
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_fp8_kernel<false>, tmA, tmW, tmWs, p);
+  if (a.gated)
+    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
+  else
+    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
+  return cudaGetLastError();
 }
 
 }  // namespace moe
