@@ -389,7 +389,8 @@ def run_native(args):
                          "algorithmic_bytes": algo["gate_up_bytes"],
                          "algorithmic_flops": algo["gate_up_flops"],
                          "launch_ms": gemm_ms, "peak_source": peaks["source"]},
-            "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / ms,
+            "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / head_ms,
+                              "frac_eager": step_roof_ms / ms,
                               "algorithmic_bytes": algo["step_bytes"],
                               "algorithmic_flops": algo["step_flops"],
                               "touched_experts": algo["touched_experts"]},
