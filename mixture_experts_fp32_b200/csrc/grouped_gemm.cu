@@ -90,7 +90,9 @@ template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmAs,
-                        const __grid_constant__ CUtensorMap tmB, const KParams p) {
+                        const __grid_constant__ CUtensorMap tmB16,
+                        const __grid_constant__ CUtensorMap tmB32,
+                        const __grid_constant__ CUtensorMap tmB64, const KParams p) {
   using C = Cfg<GATED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -122,7 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmAs);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmB16);
+    tma_prefetch_desc(&tmB32);
+    tma_prefetch_desc(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
@@ -182,8 +186,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(a_dst, am, kb * BK, arow, fb, pol_a);
           if (GATED) tma_load_2d(a_dst + BM * BK * 2, am, kb * BK, arow + up, fb, pol_a);
           const uint32_t b_dst = smem_u32(b_smem + stage * C::B_BYTES);
-          for (int nb = 0; nb < ti.n_mma / 16; ++nb)
-            tma_load_2d(b_dst + nb * 16 * BK * 2, &tmB, kb * BK, ti.row0 + nb * 16, fb, pol_b);
+          // the tile's rows in at most three boxes (64 / 32 / 16 rows): one thread
+          // issues every copy, and a copy per 16 rows left it behind the weight stream
+          for (int r = 0; r < ti.n_mma;) {
+            const int left = ti.n_mma - r;
+            const int box = left >= 64 ? 64 : left >= 32 ? 32 : 16;
+            const CUtensorMap* bm = box == 64 ? &tmB64 : box == 32 ? &tmB32 : &tmB16;
+            tma_load_2d(b_dst + r * BK * 2, bm, kb * BK, ti.row0 + r, fb, pol_b);
+            r += box;
+          }
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -339,7 +350,7 @@ cudaError_t prepare_grouped_gemm_kernels() {
 }
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
-  CUtensorMap tmA, tmAs, tmB;
+  CUtensorMap tmA, tmAs, tmB16, tmB32, tmB64;
   const uint64_t rows_routed = (uint64_t)a.E * a.rows_per_expert;
   if (!make_map_bf16(&tmA, a.a_routed, a.K_routed, rows_routed, BM)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
@@ -349,7 +360,10 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   } else {
     tmAs = tmA;
   }
-  if (!make_map_bf16(&tmB, a.b, a.K_ld, (uint64_t)a.R_cap, 16)) return cudaErrorInvalidValue;
+  if (!make_map_bf16(&tmB16, a.b, a.K_ld, (uint64_t)a.R_cap, 16) ||
+      !make_map_bf16(&tmB32, a.b, a.K_ld, (uint64_t)a.R_cap, 32) ||
+      !make_map_bf16(&tmB64, a.b, a.K_ld, (uint64_t)a.R_cap, 64))
+    return cudaErrorInvalidValue;
 
   KParams p;
   p.group_offsets = a.group_offsets;
@@ -368,11 +382,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
   if (a.gated) {
-    grouped_gemm_kernel<true><<<a.num_ctas, kThreads, Cfg<true>::SMEM_BYTES, st>>>(tmA, tmAs, tmB,
-                                                                                   p);
+    grouped_gemm_kernel<true><<<a.num_ctas, kThreads, Cfg<true>::SMEM_BYTES, st>>>(
+        tmA, tmAs, tmB16, tmB32, tmB64, p);
   } else {
-    grouped_gemm_kernel<false><<<a.num_ctas, kThreads, Cfg<false>::SMEM_BYTES, st>>>(tmA, tmAs,
-                                                                                     tmB, p);
+    grouped_gemm_kernel<false><<<a.num_ctas, kThreads, Cfg<false>::SMEM_BYTES, st>>>(
+        tmA, tmAs, tmB16, tmB32, tmB64, p);
   }
   return cudaGetLastError();
 }
