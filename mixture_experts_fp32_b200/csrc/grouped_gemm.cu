@@ -43,7 +43,9 @@ template <bool GATED>
 struct Cfg {
   static constexpr int A_BYTES = (GATED ? 2 : 1) * BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGES = GATED ? 4 : 6;
+  // down: one weight box per stage, so more stages keep enough HBM bytes in flight
+  // (7 x 32 KB + 3 KB fills the 227 KB a CTA may have)
+  static constexpr int STAGES = GATED ? 4 : 7;
   static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
   static constexpr int SMEM_BYTES = DATA_BYTES + 1024 + 2048;
 };
