@@ -151,6 +151,38 @@ moe_status moe_forward(moe_plan_t plan, const moe_weights *weights, const void *
                        const uint8_t *valid, int T, int k, void *out, void *workspace,
                        size_t ws_bytes, void *stream, moe_debug *dbg);
 
+/* Tensor-parallel MoE (DP Attention and TBO for DeepSeek-V4 on MI355X,
+ * introduction: DP attention in front of a TP MoE joined by all_gather /
+ * reduce_scatter).  Each of n ranks holds a 1/n share of every expert's
+ * intermediate dimension (a plan with inter = I/n, shared_inter = Is/n, and
+ * the matching rows of w_gate_up and columns of w_down), runs the layer on the
+ * all-gathered rows T = n * rows_per_rank, and its contributions are summed.
+ *
+ * moe_forward_scatter is the forward pass whose combine writes each token's
+ * fp32 sum (this rank's share, routed + shared, not rounded; padding rows
+ * +0.0) directly into the receive slab of the rank that owns the token:
+ *   token t -> dst[t / rows_per_rank] + (slot * rows_per_rank + t % rows_per_rank) * H
+ * so the slab of owner r is [n_dst][rows_per_rank][H] fp32 with one row block
+ * per contributing rank, and `slot` is this rank's index.  dst is a host
+ * array of n_dst (1..8) device pointers, 16-byte aligned; they may point into
+ * other GPUs' memory (peer-mapped: the kernel only stores to them), which
+ * makes the combine carry the reduce-scatter's data movement.  With n_dst = 1,
+ * rows_per_rank = T, slot = 0 it writes the plain fp32 partial [T, H].
+ * Requires n_dst * rows_per_rank == T and 0 <= slot < n_dst.  Completion on
+ * this stream says nothing about the other ranks: the owner must know that
+ * every contributor's forward has finished (a barrier) before reducing.
+ *
+ * moe_reduce_partials is the owner's half: out[t] = bf16(sum over g = 0..n_slots-1
+ * of slots[g][t]), in that order, rounded once; rows with valid[t] == 0 get
+ * +0.0.  slots: fp32 [n_slots][rows][H] (device), valid: uint8 [rows] or NULL,
+ * out: bf16 [rows][H]; H a multiple of 8, pointers 16-byte aligned. */
+moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights *weights, const void *hidden,
+                               const uint8_t *valid, int T, int k, float *const *dst, int n_dst,
+                               int rows_per_rank, int slot, void *workspace, size_t ws_bytes,
+                               void *stream, moe_debug *dbg);
+moe_status moe_reduce_partials(const float *slots, int n_slots, int rows, int H,
+                               const uint8_t *valid, void *out, void *stream);
+
 /* Routing only, from given fp32 logits [T, E] (device): the top-k selection,
  * weights, per-expert offsets and permutation exactly as moe_forward computes
  * them.  Outputs as in moe_debug (topk_ids, topk_w [T,k]; perm [T*k];

@@ -32,8 +32,10 @@ MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")
 
 EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
+            "moe_forward_scatter", "moe_reduce_partials",
             "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
             "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string")
+MAX_TP_RANKS = 8
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
 
@@ -92,6 +94,12 @@ def load():
     L.moe_forward.argtypes = [_vp, ctypes.POINTER(moe_weights), _vp, _vp, _c_int, _c_int, _vp, _vp,
                               ctypes.c_size_t, _vp, ctypes.POINTER(moe_debug)]
     L.moe_forward.restype = _c_int
+    L.moe_forward_scatter.argtypes = [_vp, ctypes.POINTER(moe_weights), _vp, _vp, _c_int, _c_int,
+                                      ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _vp,
+                                      ctypes.c_size_t, _vp, ctypes.POINTER(moe_debug)]
+    L.moe_forward_scatter.restype = _c_int
+    L.moe_reduce_partials.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]
+    L.moe_reduce_partials.restype = _c_int
     L.moe_route_from_logits.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
                                         ctypes.c_size_t, _vp]
     L.moe_route_from_logits.restype = _c_int
@@ -182,6 +190,24 @@ def moe_forward(plan, weights: moe_weights, hidden, valid, T: int, k: int, out, 
     _check(st, "moe_forward")
 
 
+def moe_forward_scatter(plan, weights: moe_weights, hidden, valid, T: int, k: int, dst,
+                        rows_per_rank: int, slot: int, workspace, ws_bytes: int, stream=None,
+                        dbg: moe_debug | None = None) -> None:
+    """dst: a sequence of device addresses (or tensors) of the owners' receive slabs."""
+    arr = (_vp * len(dst))(*[_addr(d) for d in dst])
+    st = load().moe_forward_scatter(plan, ctypes.byref(weights), _addr(hidden), _addr(valid), T, k,
+                                    arr, len(dst), rows_per_rank, slot, _addr(workspace),
+                                    ws_bytes, _stream(stream),
+                                    None if dbg is None else ctypes.byref(dbg))
+    _check(st, "moe_forward_scatter")
+
+
+def moe_reduce_partials(slots, n_slots: int, rows: int, H: int, valid, out, stream=None) -> None:
+    st = load().moe_reduce_partials(_addr(slots), n_slots, rows, H, _addr(valid), _addr(out),
+                                    _stream(stream))
+    _check(st, "moe_reduce_partials")
+
+
 def moe_route_from_logits(plan, logits, valid, T: int, k: int, topk_ids, topk_w, perm, offsets,
                           workspace, ws_bytes: int, stream=None) -> None:
     st = load().moe_route_from_logits(plan, _addr(logits), _addr(valid), T, k, _addr(topk_ids),
@@ -233,6 +259,11 @@ class Plan:
     def forward(self, weights: moe_weights, hidden, valid, k: int, out, stream=None, dbg=None):
         moe_forward(self.handle, weights, hidden, valid, hidden.shape[0], k, out, self.workspace,
                     self.ws_bytes, stream, dbg)
+
+    def forward_scatter(self, weights: moe_weights, hidden, valid, k: int, dst,
+                        rows_per_rank: int, slot: int, stream=None, dbg=None):
+        moe_forward_scatter(self.handle, weights, hidden, valid, hidden.shape[0], k, dst,
+                            rows_per_rank, slot, self.workspace, self.ws_bytes, stream, dbg)
 
     def route_from_logits(self, logits, valid, k: int, topk_ids, topk_w, perm, offsets,
                           stream=None):

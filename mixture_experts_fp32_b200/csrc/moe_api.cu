@@ -185,20 +185,23 @@ MOE_EXPORT moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns
   return MOE_OK;
 }
 
-MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const void* hidden,
-                                  const uint8_t* valid, int T, int k, void* out, void* workspace,
-                                  size_t ws_bytes, void* stream, moe_debug* dbg) {
+// The forward pass; `co` says where the combine writes (the bf16 output, or
+// fp32 tensor-parallel partial rows).  Argument checks common to both entry
+// points are here; each entry point checks its own output arguments first.
+static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const void* hidden,
+                               const uint8_t* valid, int T, int k, const moe::CombineOut& co,
+                               void* workspace, size_t ws_bytes, void* stream, moe_debug* dbg) {
   moe_status s = check_common(plan, T, k, workspace, ws_bytes);
   if (s != MOE_OK) return s;
   if (wts == nullptr) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   const moe_config& c = plan->cfg;
   const int S = c.num_shared;
-  if (hidden == nullptr || out == nullptr || wts->router_w == nullptr ||
-      wts->w_gate_up == nullptr || wts->w_down == nullptr)
+  if (hidden == nullptr || wts->router_w == nullptr || wts->w_gate_up == nullptr ||
+      wts->w_down == nullptr)
     return MOE_ERR_INVALID_ARG;
   if (S && (wts->ws_gate_up == nullptr || wts->ws_down == nullptr)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(hidden) || !aligned16(out) || !aligned16(wts->router_w) ||
+  if (!aligned16(hidden) || !aligned16(wts->router_w) ||
       !aligned16(wts->w_gate_up) || !aligned16(wts->w_down) ||
       (S && (!aligned16(wts->ws_gate_up) || !aligned16(wts->ws_down))))
     return MOE_ERR_INVALID_ARG;
@@ -308,8 +311,7 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
     if (s != MOE_OK) return s;
     record(dbg, 6, st);
 
-    s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S,
-                                         static_cast<__nv_bfloat16*>(out), st));
+    s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S, co, st));
   } else {
     moe::GroupedGemmFp8Args fa;
     memset(&fa, 0, sizeof(fa));
@@ -367,8 +369,7 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
     if (s != MOE_OK) return s;
     record(dbg, 6, st);
 
-    s = check_launch(moe::launch_combine_bf16y(y16, H, inv, w, valid, T, k, S,
-                                               static_cast<__nv_bfloat16*>(out), st));
+    s = check_launch(moe::launch_combine_bf16y(y16, H, inv, w, valid, T, k, S, co, st));
   }
   if (s != MOE_OK) return s;
   record(dbg, 7, st);
@@ -387,6 +388,46 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
       return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const void* hidden,
+                                  const uint8_t* valid, int T, int k, void* out, void* workspace,
+                                  size_t ws_bytes, void* stream, moe_debug* dbg) {
+  if (out == nullptr || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  moe::CombineOut co;
+  memset(&co, 0, sizeof(co));
+  co.bf16 = static_cast<__nv_bfloat16*>(out);
+  return forward_impl(plan, wts, hidden, valid, T, k, co, workspace, ws_bytes, stream, dbg);
+}
+
+MOE_EXPORT moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights* wts,
+                                          const void* hidden, const uint8_t* valid, int T, int k,
+                                          float* const* dst, int n_dst, int rows_per_rank,
+                                          int slot, void* workspace, size_t ws_bytes,
+                                          void* stream, moe_debug* dbg) {
+  if (dst == nullptr || n_dst < 1 || n_dst > moe::kMaxTpRanks || rows_per_rank < 1 ||
+      (long long)n_dst * rows_per_rank != T || slot < 0 || slot >= n_dst)
+    return MOE_ERR_INVALID_ARG;
+  moe::CombineOut co;
+  memset(&co, 0, sizeof(co));
+  for (int r = 0; r < n_dst; ++r) {
+    if (dst[r] == nullptr || !aligned16(dst[r])) return MOE_ERR_INVALID_ARG;
+    co.dst[r] = dst[r];
+  }
+  co.rows_per_rank = rows_per_rank;
+  co.slot = slot;
+  return forward_impl(plan, wts, hidden, valid, T, k, co, workspace, ws_bytes, stream, dbg);
+}
+
+MOE_EXPORT moe_status moe_reduce_partials(const float* slots, int n_slots, int rows, int H,
+                                          const uint8_t* valid, void* out, void* stream) {
+  if (slots == nullptr || out == nullptr || n_slots < 1 || n_slots > moe::kMaxTpRanks ||
+      rows < 0 || H <= 0 || H % 8 != 0 || !aligned16(slots) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  return check_launch(moe::launch_reduce_slots(slots, n_slots, rows, H, valid,
+                                               static_cast<__nv_bfloat16*>(out),
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 MOE_EXPORT moe_status moe_route_from_logits(moe_plan_t plan, const float* logits,

@@ -15,6 +15,17 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 constexpr int kRouterSplitMax = 16;
+constexpr int kMaxTpRanks = 8;
+
+// Where the combine writes token t's result: the layer's bf16 output row, or
+// (tensor-parallel partial) an fp32 row in the receive slab of the rank that
+// owns t: dst[t / rows_per_rank] + (slot * rows_per_rank + t % rows_per_rank) * H.
+struct CombineOut {
+  __nv_bfloat16* bf16;              // non-null: bf16 [T, H]
+  float* dst[kMaxTpRanks];          // otherwise: one slab pointer per owning rank
+  int rows_per_rank;
+  int slot;
+};
 
 // ------------------------------------------------------------------ host side
 
@@ -74,7 +85,7 @@ cudaError_t launch_quant_gather(const __nv_bfloat16* x, const uint8_t* valid, in
                                 int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st);
 cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
-                                 const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                                 const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                                  cudaStream_t st);
 cudaError_t prepare_grouped_gemm_fp8_kernels();
 
@@ -100,8 +111,11 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_tok
                                int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st);
 cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
-                           const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                           const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                            cudaStream_t st);
+// out[t] = bf16(sum over slots g ascending of slots[g][t]); rows with valid[t] == 0 -> +0.0
+cudaError_t launch_reduce_slots(const float* slots, int n_slots, int rows, int H,
+                                const uint8_t* valid, __nv_bfloat16* out, cudaStream_t st);
 cudaError_t prepare_grouped_gemm_kernels();
 const moe_config* plan_config(const moe_plan_s* plan);
 void router_split_plan(int T, int E, int H, int num_sms, int* splits, int* kb_per_split);

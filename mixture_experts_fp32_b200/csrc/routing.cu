@@ -13,7 +13,13 @@
 //   y in fp32, summed in fp32 in ascending j, shared expert last; padding rows get +0.0
 //   (the combine phase, [SGLang] MoE 모델을 위한 Single Batch Overlap 기법,
 //   §들어가며; the fused shared expert, Step3 推論最適化 (MI308X vs H20),
-//   §最適化技術).
+//   §最適化技術).  For tensor parallelism the same sum (this rank's share of the
+//   intermediate dimension) is written unrounded in fp32 straight into the
+//   receive slab of the rank that owns the token, possibly another GPU's memory
+//   (plain stores), which is the data movement of the reduce-scatter; the owner
+//   then sums its slab in rank order and rounds once (reduce_slots_kernel)
+//   (TP MoE with all_gather / reduce_scatter, DP Attention and TBO for
+//   DeepSeek-V4 on MI355X, introduction).
 #include <cuda_fp8.h>
 
 #include "moe_internal.cuh"
@@ -301,13 +307,12 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* y8, float (&v)[8]) {
   }
 }
 
-template <typename YT>
+template <typename YT, bool F32OUT>
 __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, int H,
                                                       const int* __restrict__ inv,
                                                       const float* __restrict__ w,
                                                       const uint8_t* __restrict__ valid, int T,
-                                                      int k, int S,
-                                                      __nv_bfloat16* __restrict__ out) {
+                                                      int k, int S, const CombineOut co) {
   __shared__ int rows[kMaxTopK + 1];
   __shared__ float wts[kMaxTopK];
   const int ks = k + S;
@@ -317,7 +322,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
     if (threadIdx.x < ks) rows[threadIdx.x] = ok ? inv[(size_t)t * ks + threadIdx.x] : -1;
     if (threadIdx.x < k) wts[threadIdx.x] = ok ? w[(size_t)t * k + threadIdx.x] : 0.f;
     __syncthreads();
-    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+    uint4* dst16 = nullptr;
+    float4* dst32 = nullptr;
+    if (F32OUT) {
+      const int owner = t / co.rows_per_rank, lt = t - owner * co.rows_per_rank;
+      dst32 = reinterpret_cast<float4*>(co.dst[owner] +
+                                        ((size_t)co.slot * co.rows_per_rank + lt) * H);
+    } else {
+      dst16 = reinterpret_cast<uint4*>(co.bf16 + (size_t)t * H);
+    }
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
@@ -336,13 +349,50 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
           for (int i = 0; i < 8; ++i) acc[i] += yv[i];
         }
       }
+      if (F32OUT) {
+        dst32[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst32[2 * v + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+        uint4 o;
+        __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        dst16[v] = o;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Owner side of the tensor-parallel reduction: the slab holds one fp32 partial
+// row per rank for each of this rank's rows; they are summed in rank order (the
+// same order on every owner) and rounded once to bf16.
+__global__ void __launch_bounds__(256) reduce_slots_kernel(const float* __restrict__ slots,
+                                                           int n_slots, int rows, int H,
+                                                           const uint8_t* __restrict__ valid,
+                                                           __nv_bfloat16* __restrict__ out) {
+  const int nv = H / 8;
+  const size_t slab = (size_t)rows * H;
+  for (int t = blockIdx.x; t < rows; t += gridDim.x) {
+    const bool ok = valid == nullptr || valid[t];
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (ok) {
+        for (int g = 0; g < n_slots; ++g) {
+          const float4* src =
+              reinterpret_cast<const float4*>(slots + g * slab + (size_t)t * H) + 2 * v;
+          const float4 a = src[0], b = src[1];
+          acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+          acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        }
+      }
       uint4 o;
       __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
       for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
       dst[v] = o;
     }
-    __syncthreads();
   }
 }
 
@@ -446,20 +496,34 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_tok
 }
 
 cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
-                           const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                           const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                            cudaStream_t st) {
   int grid = T < 148 * 16 ? T : 148 * 16;
   if (grid < 1) grid = 1;
-  combine_kernel<float><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  if (out.bf16 != nullptr)
+    combine_kernel<float, false><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  else
+    combine_kernel<float, true><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
-                                 const uint8_t* valid, int T, int k, int S, __nv_bfloat16* out,
+                                 const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                                  cudaStream_t st) {
   int grid = T < 148 * 16 ? T : 148 * 16;
   if (grid < 1) grid = 1;
-  combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  if (out.bf16 != nullptr)
+    combine_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  else
+    combine_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_slots(const float* slots, int n_slots, int rows, int H,
+                                const uint8_t* valid, __nv_bfloat16* out, cudaStream_t st) {
+  int grid = rows < 148 * 16 ? rows : 148 * 16;
+  if (grid < 1) grid = 1;
+  reduce_slots_kernel<<<grid, 256, 0, st>>>(slots, n_slots, rows, H, valid, out);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,211 @@
+"""Tensor-parallel MoE behind data-parallel attention ranks.
+
+DP attention in front of a TP MoE, joined by standard collectives (DP Attention and
+TBO for DeepSeek-V4 on MI355X, introduction): every rank all_gathers the hidden rows of
+all DP ranks, computes the whole layer for them with its 1/n share of every expert's
+intermediate dimension, and the n partial outputs are summed back to the rank that owns
+each row.  Splitting the intermediate dimension is exact: with gate/up rows and down
+columns split alike, sum over shards of the shard layers equals the layer (the 1x128
+activation groups of the FP8 path stay whole when I/n is a multiple of 128).  Routing is
+computed by every rank from the same gathered rows and the same router, so all ranks
+agree without exchanging it.
+
+Two ways to return the partial sums:
+  * fused: the library's combine writes each row's fp32 partial straight into the
+    owner's receive slab (symmetric memory, peer pointers; `moe_forward_scatter`), a
+    device barrier (bounded) tells every owner that all contributions have landed, and
+    the owner sums its slab in rank order and rounds once (`moe_reduce_partials`);
+  * nccl: the fp32 partial [n * rows, H] goes through NCCL's reduce_scatter, then is
+    rounded by `moe_reduce_partials` with one slot.
+The fused form needs no copy of the partial and sums in the same order on every owner.
+
+Two micro-batches (TBO at the collective boundaries, same page, §最大の見どころ): the
+local rows are split in two; the all_gather of the second runs on a communication stream
+while the first computes, and (nccl form) the first's reduce_scatter runs while the
+second computes.
+
+Row ownership: gathered row t belongs to rank t // rows, local row t % rows.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional
+
+import torch
+
+import mixture_experts_fp32_b200 as moe
+
+
+def shard_weights(full: Dict[str, Optional[torch.Tensor]], n: int, r: int, *, I: int, Is: int,
+                  fp8: bool) -> Dict[str, Optional[torch.Tensor]]:
+    """Rank r's share (1/n of every expert's intermediate dimension) of the layer's
+    weights, as contiguous tensors on the same device.
+
+    w_gate_up [E, 2I, H]: gate rows [r I/n, (r+1) I/n) and the same up rows (offset I);
+    w_down [E, H, I]: the same columns; FP8 block scales [E, 2I/128, H/128] and
+    [E, H/128, I/128] follow their 128-blocks; the shared expert likewise with Is."""
+    if I % (128 * n) or (Is and Is % (128 * n)):
+        raise ValueError("each rank's share of the intermediate dimensions must be a multiple "
+                         "of 128 (the GEMM tiles and the FP8 blocks)")
+    i0, i1 = r * I // n, (r + 1) * I // n
+    out = {"router_w": full["router_w"], "router_b": full.get("router_b")}
+    wgu = full["w_gate_up"]
+    out["w_gate_up"] = torch.cat([wgu[:, i0:i1], wgu[:, I + i0:I + i1]], dim=1).contiguous()
+    out["w_down"] = full["w_down"][:, :, i0:i1].contiguous()
+    if fp8:
+        b0, b1, bI = i0 // 128, i1 // 128, I // 128
+        sgu = full["s_gate_up"]
+        out["s_gate_up"] = torch.cat([sgu[:, b0:b1], sgu[:, bI + b0:bI + b1]], dim=1).contiguous()
+        out["s_down"] = full["s_down"][:, :, b0:b1].contiguous()
+    if full.get("ws_gate_up") is not None:
+        j0, j1 = r * Is // n, (r + 1) * Is // n
+        ws = full["ws_gate_up"]
+        out["ws_gate_up"] = torch.cat([ws[j0:j1], ws[Is + j0:Is + j1]], dim=0).contiguous()
+        out["ws_down"] = full["ws_down"][:, j0:j1].contiguous()
+        if fp8:
+            c0, c1, cI = j0 // 128, j1 // 128, Is // 128
+            ss = full["ss_gate_up"]
+            out["ss_gate_up"] = torch.cat([ss[c0:c1], ss[cI + c0:cI + c1]], dim=0).contiguous()
+            out["ss_down"] = full["ss_down"][:, c0:c1].contiguous()
+    return out
+
+
+def make_shard_weights(sh: Dict[str, Optional[torch.Tensor]]) -> moe.moe_weights:
+    return moe.make_weights(sh["router_w"], sh.get("router_b"), sh["w_gate_up"], sh["w_down"],
+                            sh.get("s_gate_up"), sh.get("s_down"), sh.get("ws_gate_up"),
+                            sh.get("ws_down"), sh.get("ss_gate_up"), sh.get("ss_down"))
+
+
+def owner_of(t: int, rows: int):
+    """(owning rank, local row) of gathered row t."""
+    return t // rows, t % rows
+
+
+def split_rows(rows: int):
+    """The two micro-batches of a rank's rows: [0, a) and [a, rows), a = rows // 2."""
+    a = rows // 2
+    return (0, a), (a, rows)
+
+
+class TPMoE:
+    """One rank of the tensor-parallel layer.  `full` holds the whole layer's weights on
+    this rank's device (the shard is cut from it); `rows` is the number of rows each
+    DP rank contributes per micro-batch (padding rows included, marked invalid)."""
+
+    def __init__(self, full: dict, *, E: int, H: int, I: int, S: int, Is: int, k_max: int,
+                 rows: int, fp8: bool = False, fused: bool = True, group=None,
+                 barrier_timeout_ms: int = 10000):
+        import torch.distributed as dist
+        self.group = group if group is not None else dist.group.WORLD
+        self.n = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if self.n > moe.MAX_TP_RANKS:
+            raise ValueError("at most 8 tensor-parallel ranks")
+        self.H, self.rows, self.fused = H, rows, fused
+        self.timeout_ms = barrier_timeout_ms
+        self.shard = shard_weights(full, self.n, self.rank, I=I, Is=Is, fp8=fp8)
+        self.weights = make_shard_weights(self.shard)
+        dev = full["w_gate_up"].device
+        T = self.n * rows
+        self.plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
+                             inter=I // self.n, num_shared=S, shared_inter=Is // self.n if S else 0,
+                             wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16, device=dev)
+        self.x_all = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.valid_all = torch.empty(T, dtype=torch.uint8, device=dev)
+        self.step = 0
+        if fused:
+            import torch.distributed._symmetric_memory as symm
+            # two slabs, used on alternate steps: a rank may write step s+1's rows into
+            # an owner's slab only after that owner has reduced step s-1 from it, which
+            # the barrier of step s guarantees (each rank reduces s-1 before it scatters s)
+            self.slab = symm.empty(2, self.n, rows, H, dtype=torch.float32, device=dev)
+            self.handle = symm.rendezvous(self.slab, self.group)
+            base = [int(p) for p in self.handle.buffer_ptrs]
+            per = self.n * rows * H * 4
+            self.dst = [[b + par * per for b in base] for par in range(2)]
+        else:
+            self.partial = torch.empty(T, H, dtype=torch.float32, device=dev)
+            self.recv = torch.empty(rows, H, dtype=torch.float32, device=dev)
+
+    def _gather(self, x_local, valid_local):
+        import torch.distributed as dist
+        dist.all_gather_into_tensor(self.x_all, x_local, group=self.group)
+        dist.all_gather_into_tensor(self.valid_all, valid_local, group=self.group)
+
+    def _compute_and_return(self, k: int, valid_local, out_local):
+        import torch.distributed as dist
+        if self.fused:
+            par = self.step & 1
+            self.plan.forward_scatter(self.weights, self.x_all, self.valid_all, k, self.dst[par],
+                                      self.rows, self.rank)
+            self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
+            moe.moe_reduce_partials(self.slab[par], self.n, self.rows, self.H, valid_local,
+                                    out_local)
+        else:
+            self.plan.forward_scatter(self.weights, self.x_all, self.valid_all, k,
+                                      [self.partial], self.n * self.rows, 0)
+            dist.reduce_scatter_tensor(self.recv, self.partial, op=dist.ReduceOp.SUM,
+                                       group=self.group)
+            moe.moe_reduce_partials(self.recv, 1, self.rows, self.H, valid_local, out_local)
+        self.step += 1
+
+    def forward(self, x_local, valid_local, k: int, out_local):
+        """x_local bf16 [rows, H], valid_local uint8 [rows], out_local bf16 [rows, H]."""
+        self._gather(x_local, valid_local)
+        self._compute_and_return(k, valid_local, out_local)
+
+
+class TPMoETwoBatch:
+    """The two-micro-batch schedule: two TPMoE halves (one per micro-batch, each with
+    its own plan, gathered rows and slabs); the all_gather of micro-batch 1 is issued on
+    a communication stream so that it runs while micro-batch 0 computes."""
+
+    def __init__(self, full: dict, *, rows: int, **kw):
+        (a0, a1), (b0, b1) = split_rows(rows)
+        self.ranges = [(a0, a1), (b0, b1)]
+        self.halves = [TPMoE(full, rows=a1 - a0, **kw), TPMoE(full, rows=b1 - b0, **kw)]
+        self.comm = torch.cuda.Stream(device=full["w_gate_up"].device)
+
+    def forward(self, x_local, valid_local, k: int, out_local):
+        main = torch.cuda.current_stream()
+        ev = []
+        self.comm.wait_stream(main)
+        with torch.cuda.stream(self.comm):
+            for (lo, hi), half in zip(self.ranges, self.halves):
+                half._gather(x_local[lo:hi], valid_local[lo:hi])
+                e = torch.cuda.Event()
+                e.record(self.comm)
+                ev.append(e)
+        for e, (lo, hi), half in zip(ev, self.ranges, self.halves):
+            main.wait_event(e)
+            half._compute_and_return(k, valid_local[lo:hi], out_local[lo:hi])
+        main.wait_stream(self.comm)
+
+
+def tp_forward_reference(full: dict, x_rows: List[torch.Tensor], valid_rows: List[torch.Tensor],
+                         k: int, *, E, H, I, S, Is, k_max, fp8, n_shards: int):
+    """One-GPU emulation of n ranks (no process group): every shard's forward scatters
+    into every owner's slab, then each owner reduces.  Returns the owners' outputs."""
+    dev = full["w_gate_up"].device
+    rows = x_rows[0].shape[0]
+    x_all = torch.cat(x_rows)
+    v_all = torch.cat(valid_rows)
+    T = n_shards * rows
+    slabs = [torch.full((n_shards, rows, H), float("nan"), dtype=torch.float32, device=dev)
+             for _ in range(n_shards)]
+    plans = []
+    for r in range(n_shards):
+        sh = shard_weights(full, n_shards, r, I=I, Is=Is, fp8=fp8)
+        plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
+                        inter=I // n_shards, num_shared=S,
+                        shared_inter=Is // n_shards if S else 0,
+                        wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16, device=dev)
+        plan.forward_scatter(make_shard_weights(sh), x_all, v_all, k, [s for s in slabs],
+                             rows, r)
+        plans.append((plan, sh))
+    outs = []
+    for r in range(n_shards):
+        o = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+        moe.moe_reduce_partials(slabs[r], n_shards, rows, H, valid_rows[r], o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    return outs

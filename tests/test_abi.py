@@ -126,3 +126,36 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
                                          None) == moe.MOE_ERR_INVALID_ARG
     finally:
         moe.moe_plan_destroy(plan)
+
+
+def test_tensor_parallel_entry_points_reject_bad_arguments_before_launch(lib):
+    plan, ws = moe.moe_plan_create(cfg())
+    try:
+        w = moe.make_weights(0x1000, None, 0x2000, 0x3000, ws_gate_up=0x4000, ws_down=0x5000)
+        WS = 0x100000
+
+        def scatter(dst, rpr, slot, T=16):
+            arr = (ctypes.c_void_p * max(1, len(dst)))(*dst)
+            return lib.moe_forward_scatter(plan, ctypes.byref(w), 0x6000, None, T, 3, arr,
+                                           len(dst), rpr, slot, WS, ws, None, None)
+
+        assert scatter([0x7000, 0x8000], 8, 0, T=17) == moe.MOE_ERR_INVALID_ARG   # n * rpr != T
+        assert scatter([], 16, 0) == moe.MOE_ERR_INVALID_ARG                       # no owners
+        assert scatter([0x7000] * 9, 2, 0, T=18) == moe.MOE_ERR_INVALID_ARG        # > 8 ranks
+        assert scatter([0x7000, 0x8000], 8, 2) == moe.MOE_ERR_INVALID_ARG          # slot >= n
+        assert scatter([0x7000, 0x8000], 8, -1) == moe.MOE_ERR_INVALID_ARG
+        assert scatter([0x7000, 0x8008], 8, 0) == moe.MOE_ERR_INVALID_ARG          # unaligned
+        assert scatter([0x7000, 0], 8, 0) == moe.MOE_ERR_INVALID_ARG               # null owner
+        assert scatter([0x7000, 0x8000], 0, 0, T=0) == moe.MOE_ERR_INVALID_ARG     # rpr 0
+        arr = (ctypes.c_void_p * 2)(0x7000, 0x8000)
+        assert lib.moe_forward_scatter(plan, ctypes.byref(w), 0x6000, None, 16, 4, arr, 2, 8, 0,
+                                       WS, ws, None, None) == moe.MOE_ERR_INVALID_ARG  # k > max
+        red = lib.moe_reduce_partials
+        assert red(None, 2, 4, 64, None, 0x9000, None) == moe.MOE_ERR_INVALID_ARG
+        assert red(0x7000, 0, 4, 64, None, 0x9000, None) == moe.MOE_ERR_INVALID_ARG
+        assert red(0x7000, 9, 4, 64, None, 0x9000, None) == moe.MOE_ERR_INVALID_ARG
+        assert red(0x7000, 2, 4, 60, None, 0x9000, None) == moe.MOE_ERR_INVALID_ARG   # H % 8
+        assert red(0x7004, 2, 4, 64, None, 0x9000, None) == moe.MOE_ERR_INVALID_ARG   # unaligned
+        assert red(0x7000, 2, 0, 64, None, 0x9000, None) == moe.MOE_OK                 # no rows
+    finally:
+        moe.moe_plan_destroy(plan)
