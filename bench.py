@@ -450,6 +450,101 @@ def cpu_baseline(w, args):
                       f"double-precision C with OpenMP over tokens"}
 
 
+def run_tp(args):
+    """Tensor-parallel layout (--tp): the workload's rows are the all-gathered batch of N
+    DP ranks (rows T/N each); every rank holds 1/N of each expert's intermediate
+    dimension and returns its partial sums to the owners (fused into the combine, or
+    NCCL reduce_scatter with --tp-return nccl).  Whole-job valid tokens/s; the gathered
+    batch is fixed, so adding ranks is strong scaling."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_fp32_b200 as moe
+    from mixture_experts_fp32_b200 import build as lib_build
+    from mixture_experts_fp32_b200 import tp
+    import synth
+
+    ws_n, rank, local = dist_env()
+    if "MASTER_ADDR" not in os.environ:                   # one process without torchrun
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(sk.getsockname()[1]))
+        sk.close()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", rank=rank, world_size=ws_n, device_id=dev,
+                            timeout=__import__("datetime").timedelta(seconds=600))
+    layer = None
+    try:
+        if rank == 0:
+            lib_build.build()
+        dist.barrier()
+        moe.load()
+        w = workload_of(args)
+        if w.T % ws_n:
+            raise SystemExit(f"{w.T} rows do not split over {ws_n} ranks")
+        rows = w.T // ws_n
+        inp = synth.make_inputs(w)        # the same seeded layer and gathered batch on every rank
+        d = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
+        del inp
+        layer = tp.TPMoE(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is if w.S else 0, k_max=w.k,
+                         rows=rows, fp8=w.wtype == "fp8", fused=args.tp_return == "fused")
+        x_loc = d["x"][rank * rows:(rank + 1) * rows].contiguous()
+        v_loc = d["valid"][rank * rows:(rank + 1) * rows].contiguous()
+        valid_tokens = int(d["valid"].sum().item())
+        for key in ("w_gate_up", "w_down", "ws_gate_up", "ws_down", "s_gate_up", "s_down",
+                    "ss_gate_up", "ss_down"):
+            d[key] = None                                  # the shard keeps its own copy
+        torch.cuda.empty_cache()
+        out = torch.empty(rows, w.H, dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            layer.forward(x_loc, v_loc, w.k, out)
+        torch.cuda.synchronize()
+        if layer.plan.device_status() != 0:
+            raise RuntimeError("device status set during warm-up")
+        K = args.steps
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        clocks = ClockSampler(dev.index)
+        clocks.start()
+        dist.barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record()
+            layer.forward(x_loc, v_loc, w.k, out)
+            e1.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        clk = clocks.stop()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
+        ms = reduce_over_ranks(ms, "max", ws_n, dev)
+        if layer.plan.device_status() != 0:
+            raise RuntimeError("device status set during the timed steps")
+        if rank == 0:
+            print(json.dumps({
+                "metric": METRIC, "value": valid_tokens / (ms * 1e-3), "unit": "tokens/s",
+                "n_gpus": ws_n, "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": w.wtype, "data": "synthetic (Philox4x32-10, seed 0)",
+                "timing": "eager TP forward per step (all_gather, layer, partial return, reduce)",
+                "config": {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens,
+                           "rows_per_rank": rows, "H": w.H, "E": w.E, "k": w.k, "I": w.I,
+                           "S": w.S, "parallelism": f"tp{ws_n}",
+                           "partial_return": args.tp_return,
+                           "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps"},
+                "clocks": clk}))
+    finally:
+        del layer
+        torch.cuda.synchronize()
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     ws_n, rank, _ = dist_env()
     if rank != 0:
@@ -498,11 +593,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager forwards only (default: the headline is CUDA-graph replay)")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor-parallel layout over the N ranks (default workload: dp_padded)")
+    ap.add_argument("--tp-return", default="fused", choices=["fused", "nccl"])
     ap.add_argument("--experts", type=int, default=0,
                     help="override the number of routed experts (profiling on a smaller case)")
     args = ap.parse_args(argv)
+    if args.tp and args.workload == DEFAULT_WORKLOAD and "--workload" not in (argv or sys.argv):
+        args.workload = "dp_padded"
     if args.impl == "reference":
         run_reference(args)
+    elif args.tp:
+        run_tp(args)
     else:
         run_native(args)
 
