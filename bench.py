@@ -59,11 +59,10 @@ def dist_env():
 
 def launches_per_step(w) -> int:
     """Kernels one forward launches: weight split + router + top-k, the permutation
-    (1 kernel up to 1024 rows, 3 above), gather (FP8: quantise + gather), the two
-    GEMMs and the combine."""
+    (1 kernel up to 1024 rows, 3 above), the row gather (FP8: quantise-and-scatter),
+    the two GEMMs and the combine."""
     route = 1 if w.T <= 1024 else 3
-    gather = 2 if w.wtype == "fp8" else 1
-    return 3 + route + gather + 2 + 1
+    return 3 + route + 1 + 2 + 1
 
 
 def replica_seed(seed: int, rank: int) -> int:

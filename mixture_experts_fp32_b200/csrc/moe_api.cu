@@ -19,7 +19,7 @@ struct moe_plan_s {
   // byte offsets inside the workspace
   size_t off_status, off_goff, off_wsplit, off_rscratch, off_partial, off_logits, off_ids, off_w,
       off_perm,
-      off_inv, off_rowtok, off_xp, off_sx, off_xqt, off_sxt, off_h, off_sh, off_y;
+      off_inv, off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
   unsigned long long wait_limit_ns;
   int device;
   int num_sms;
@@ -154,7 +154,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   if (c.wtype == MOE_W_BF16) {
     // bf16 permuted rows and h; fp32 expert outputs
     p->off_xp = take(2 * r_cap * H);
-    p->off_sx = p->off_xqt = p->off_sxt = 0;
+    p->off_sx = 0;
     p->off_h = take(2 * r_cap * (size_t)imax);
     p->off_sh = 0;
     p->off_y = take(sizeof(float) * r_cap * H);
@@ -162,8 +162,6 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
     // e4m3 permuted rows and h with transposed 1x128 scales; bf16 expert outputs
     p->off_xp = take(r_cap * H);
     p->off_sx = take(sizeof(float) * (H / 128) * r_cap);
-    p->off_xqt = take(T * H);                             // each token quantised once
-    p->off_sxt = take(sizeof(float) * (H / 128) * T);
     p->off_h = take(r_cap * (size_t)imax);
     p->off_sh = take(sizeof(float) * ((size_t)imax / 128) * r_cap);
     p->off_y = take(2 * r_cap * H);
@@ -255,10 +253,10 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     s = check_launch(
         moe::launch_gather_rows(x, H, rowtok, goff + G, R_cap, xp, plan->num_sms, st));
   } else {
-    s = check_launch(moe::launch_quant_gather(
-        x, valid, T, H, rowtok, goff + G, R_cap, at<uint8_t>(workspace, plan->off_xqt),
-        at<float>(workspace, plan->off_sxt), at<uint8_t>(workspace, plan->off_xp),
-        at<float>(workspace, plan->off_sx), plan->num_sms, st));
+    s = check_launch(moe::launch_quant_scatter(x, valid, T, H, inv, ks,
+                                               at<uint8_t>(workspace, plan->off_xp),
+                                               at<float>(workspace, plan->off_sx),
+                                               plan->num_sms, st));
   }
   if (s != MOE_OK) return s;
   record(dbg, 4, st);

@@ -77,12 +77,11 @@ struct GroupedGemmFp8Args {
   int num_ctas;
 };
 
-// FP8: quantise every valid token once (xq_tok [T, H], sx_tok [T, H/128]), then
-// copy codes and scales into permuted order (xp [R, H], sxp [R, H/128]).
-cudaError_t launch_quant_gather(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
-                                const int* row_token, const int* total_rows, int R_cap,
-                                uint8_t* xq_tok, float* sx_tok, uint8_t* xp, float* sxp,
-                                int num_sms, cudaStream_t st);
+// FP8: quantise every valid token once (1x128 groups) and store codes and scales into
+// each of its permuted rows (xp [R, H], sxp [R, H/128]) through the inverse map inv [T, ks].
+cudaError_t launch_quant_scatter(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
+                                 const int* inv, int ks, uint8_t* xp, float* sxp, int num_sms,
+                                 cudaStream_t st);
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st);
 cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, const float* w,
                                  const uint8_t* valid, int T, int k, int S, const CombineOut& out,

@@ -291,20 +291,33 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
   }
 }
 
-// Eight consecutive expert outputs as fp32 (fp32 rows, or bf16 rows of the FP8 path).
-__device__ __forceinline__ void load8(const float* y8, float (&v)[8]) {
-  const float4 a = reinterpret_cast<const float4*>(y8)[0];
-  const float4 b = reinterpret_cast<const float4*>(y8)[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+// Eight consecutive expert outputs as loaded: two 16-byte vectors of fp32 rows, or
+// one of bf16 rows (FP8 path), widened to fp32 when summed.
+template <typename YT> struct Vec8;
+template <> struct Vec8<float> {
+  float4 a, b;
+};
+template <> struct Vec8<__nv_bfloat16> {
+  uint4 r;
+};
+__device__ __forceinline__ Vec8<float> ld8(const float* y8) {
+  Vec8<float> v;
+  v.a = reinterpret_cast<const float4*>(y8)[0];
+  v.b = reinterpret_cast<const float4*>(y8)[1];
+  return v;
 }
-__device__ __forceinline__ void load8(const __nv_bfloat16* y8, float (&v)[8]) {
-  const uint4 raw = *reinterpret_cast<const uint4*>(y8);
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __low2float(p[i]);
-    v[2 * i + 1] = __high2float(p[i]);
-  }
+__device__ __forceinline__ Vec8<__nv_bfloat16> ld8(const __nv_bfloat16* y8) {
+  Vec8<__nv_bfloat16> v;
+  v.r = *reinterpret_cast<const uint4*>(y8);
+  return v;
+}
+__device__ __forceinline__ float elem8(const Vec8<float>& v, int i) {
+  return i < 4 ? (i == 0 ? v.a.x : i == 1 ? v.a.y : i == 2 ? v.a.z : v.a.w)
+               : (i == 4 ? v.b.x : i == 5 ? v.b.y : i == 6 ? v.b.z : v.b.w);
+}
+__device__ __forceinline__ float elem8(const Vec8<__nv_bfloat16>& v, int i) {
+  const uint32_t w = i < 2 ? v.r.x : i < 4 ? v.r.y : i < 6 ? v.r.z : v.r.w;
+  return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));   // bf16 -> fp32 is exact
 }
 
 template <typename YT, bool F32OUT>
@@ -326,27 +339,39 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
     float4* dst32 = nullptr;
     if (F32OUT) {
       const int owner = t / co.rows_per_rank, lt = t - owner * co.rows_per_rank;
-      dst32 = reinterpret_cast<float4*>(co.dst[owner] +
-                                        ((size_t)co.slot * co.rows_per_rank + lt) * H);
+      float* base = co.dst[0];
+#pragma unroll
+      for (int r = 1; r < kMaxTpRanks; ++r)
+        if (owner == r) base = co.dst[r];
+      dst32 = reinterpret_cast<float4*>(base + ((size_t)co.slot * co.rows_per_rank + lt) * H);
     } else {
       dst16 = reinterpret_cast<uint4*>(co.bf16 + (size_t)t * H);
     }
     for (int v = threadIdx.x; v < nv; v += blockDim.x) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (ok) {
-        for (int j = 0; j < k; ++j) {
-          const int r = rows[j];
-          if (r < 0) continue;
-          float yv[8];
-          load8(y + (size_t)r * H + (size_t)v * 8, yv);
+        // every row's vector is requested before the sums (one round trip, not k+S),
+        // and the sums keep their order: j ascending, then the shared expert
+        // (named registers rather than an array, which the compiler put in local memory)
+        static_assert(kMaxTopK == 8, "one register set per possible row below");
+        const YT* yv = y + (size_t)v * 8;
+#define MOE_LD(J) \
+  Vec8<YT> r##J;  \
+  if (J < ks) r##J = ld8(yv + (size_t)rows[J] * H);
+        MOE_LD(0) MOE_LD(1) MOE_LD(2) MOE_LD(3) MOE_LD(4) MOE_LD(5) MOE_LD(6) MOE_LD(7) MOE_LD(8)
+#undef MOE_LD
+#define MOE_FMA(J)                                                                 \
+  if (J < k) {                                                                     \
+    _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] =                         \
+        fmaf(wts[J], elem8(r##J, i), acc[i]);                                      \
+  }
+        MOE_FMA(0) MOE_FMA(1) MOE_FMA(2) MOE_FMA(3) MOE_FMA(4) MOE_FMA(5) MOE_FMA(6) MOE_FMA(7)
+#undef MOE_FMA
+        if (S) {                                       // the shared expert's row, slot k
+          const Vec8<YT>& rs = k == 1 ? r1 : k == 2 ? r2 : k == 3 ? r3 : k == 4 ? r4
+                             : k == 5 ? r5 : k == 6 ? r6 : k == 7 ? r7 : r8;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(wts[j], yv[i], acc[i]);
-        }
-        if (S && rows[k] >= 0) {
-          float yv[8];
-          load8(y + (size_t)rows[k] * H + (size_t)v * 8, yv);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += yv[i];
+          for (int i = 0; i < 8; ++i) acc[i] += elem8(rs, i);
         }
       }
       if (F32OUT) {
@@ -396,58 +421,64 @@ __global__ void __launch_bounds__(256) reduce_slots_kernel(const float* __restri
   }
 }
 
-// FP8 path, activation quantisation of each valid token once: e4m3 codes of
-// x[t] with one scale per 1x128 group, s = amax / 448 (1 when amax = 0),
-// q = e4m3_rne_sat(x / s), both fp32 divisions correctly rounded.  A warp owns
-// one group (4 values a lane).  Scales are row-major, sx[t][g].
-__global__ void __launch_bounds__(256) quant_tokens_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           const uint8_t* __restrict__ valid,
-                                                           int T, int H,
-                                                           uint8_t* __restrict__ xq,
-                                                           float* __restrict__ sx) {
+// FP8 path, activation quantisation: a warp takes up to four 1x128 groups of one
+// valid token (their loads issued together), computes for each s = amax / 448 (1 if
+// amax = 0) and the e4m3 codes of x / s (fp32 division, round to nearest even,
+// saturating), once per token, and stores codes and scale straight into every
+// permuted row the token occupies (its k routed rows and the shared one, from the
+// inverse permutation): the GEMM's activation rows are written once, with no
+// per-token copy to gather from.
+constexpr int kQuantGroupsPerWarp = 4;
+
+__global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            const uint8_t* __restrict__ valid,
+                                                            int T, int H,
+                                                            const int* __restrict__ inv, int ks,
+                                                            uint8_t* __restrict__ xp,
+                                                            float* __restrict__ sxp) {
   const int lane = threadIdx.x & 31;
   const int groups = H / 128;
+  const int chunks = (groups + kQuantGroupsPerWarp - 1) / kQuantGroupsPerWarp;
   const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
-  for (long long wg = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-       wg < (long long)T * groups; wg += nwarps) {
-    const int t = (int)(wg / groups), g = (int)(wg - (long long)t * groups);
+  for (long long wc = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+       wc < (long long)T * chunks; wc += nwarps) {
+    const int t = (int)(wc / chunks);
+    const int g0 = (int)(wc - (long long)t * chunks) * kQuantGroupsPerWarp;
     if (valid != nullptr && !valid[t]) continue;
-    const uint2 raw =
-        *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)g * 128 + lane * 4);
-    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
-    float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    const int ng = min(kQuantGroupsPerWarp, groups - g0);
+    uint2 raw[kQuantGroupsPerWarp];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-    const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-    uint32_t packed = 0;
+    for (int u = 0; u < kQuantGroupsPerWarp; ++u)
+      if (u < ng)
+        raw[u] = *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)(g0 + u) * 128 +
+                                                 lane * 4);
+    int rows[kMaxTopK + 1];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
-                << (8 * i);
-    *reinterpret_cast<uint32_t*>(xq + (size_t)t * H + (size_t)g * 128 + lane * 4) = packed;
-    if (lane == 0) sx[(size_t)t * groups + g] = s;
-  }
-}
-
-// x_perm[r] = xq[row_token[r]] and its scale row, 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_fp8_rows_kernel(const uint8_t* __restrict__ xq,
-                                                              const float* __restrict__ sx,
-                                                              int H,
-                                                              const int* __restrict__ row_token,
-                                                              const int* __restrict__ total_rows,
-                                                              uint8_t* __restrict__ xp,
-                                                              float* __restrict__ sxp) {
-  const int R = *total_rows;
-  const int nv = H / 16, groups = H / 128;
-  for (int r = blockIdx.x; r < R; r += gridDim.x) {
-    const int t = row_token[r];
-    const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * H);
-    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * H);
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) dst[v] = src[v];
-    for (int g = threadIdx.x; g < groups; g += blockDim.x)
-      sxp[(size_t)r * groups + g] = sx[(size_t)t * groups + g];
+    for (int j = 0; j < kMaxTopK + 1; ++j) rows[j] = j < ks ? inv[(size_t)t * ks + j] : -1;
+#pragma unroll
+    for (int u = 0; u < kQuantGroupsPerWarp; ++u) {
+      if (u >= ng) break;
+      const int g = g0 + u;
+      const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw[u].x);
+      const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw[u].y);
+      const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
+      float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
+                  << (8 * i);
+#pragma unroll
+      for (int j = 0; j < kMaxTopK + 1; ++j) {
+        const int r = rows[j];
+        if (r < 0) continue;
+        *reinterpret_cast<uint32_t*>(xp + (size_t)r * H + (size_t)g * 128 + lane * 4) = packed;
+        if (lane == 0) sxp[(size_t)r * groups + g] = s;
+      }
+    }
   }
 }
 
@@ -527,20 +558,15 @@ cudaError_t launch_reduce_slots(const float* slots, int n_slots, int rows, int H
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_gather(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
-                                const int* row_token, const int* total_rows, int R_cap,
-                                uint8_t* xq_tok, float* sx_tok, uint8_t* xp, float* sxp,
-                                int num_sms, cudaStream_t st) {
-  const long long warps = (long long)T * (H / 128);
+cudaError_t launch_quant_scatter(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
+                                 const int* inv, int ks, uint8_t* xp, float* sxp, int num_sms,
+                                 cudaStream_t st) {
+  const int chunks = (H / 128 + kQuantGroupsPerWarp - 1) / kQuantGroupsPerWarp;
+  const long long warps = (long long)T * chunks;
   long long g1 = (warps + 7) / 8;
   if (g1 > (long long)num_sms * 16) g1 = (long long)num_sms * 16;
-  quant_tokens_kernel<<<(int)g1, 256, 0, st>>>(x, valid, T, H, xq_tok, sx_tok);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  int grid = num_sms * 8;
-  if (grid > R_cap) grid = R_cap;
-  if (grid < 1) grid = 1;
-  gather_fp8_rows_kernel<<<grid, 256, 0, st>>>(xq_tok, sx_tok, H, row_token, total_rows, xp, sxp);
+  if (g1 < 1) g1 = 1;
+  quant_scatter_kernel<<<(int)g1, 256, 0, st>>>(x, valid, T, H, inv, ks, xp, sxp);
   return cudaGetLastError();
 }
 
