@@ -450,9 +450,10 @@ def cpu_baseline(w, args):
 
 
 def run_tp(args):
-    """Tensor-parallel layout (--tp): the workload's rows are the all-gathered batch of N
-    DP ranks (rows T/N each); every rank holds 1/N of each expert's intermediate
-    dimension and returns its partial sums to the owners (fused into the combine, or
+    """Tensor- or expert-parallel layout (--tp, --tp-layout tp|ep): the workload's rows
+    are the all-gathered batch of N DP ranks (rows T/N each); every rank holds 1/N of
+    each expert's intermediate dimension (tp) or 1/N of the experts and of the shared
+    expert (ep) and returns its partial sums to the owners (fused into the combine, or
     NCCL reduce_scatter with --tp-return nccl).  Whole-job valid tokens/s; the gathered
     batch is fixed, so adding ranks is strong scaling."""
     import socket
@@ -489,7 +490,8 @@ def run_tp(args):
         d = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
         del inp
         layer = tp.TPMoE(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is if w.S else 0, k_max=w.k,
-                         rows=rows, fp8=w.wtype == "fp8", fused=args.tp_return == "fused")
+                         rows=rows, fp8=w.wtype == "fp8", fused=args.tp_return == "fused",
+                         layout=args.tp_layout)
         x_loc = d["x"][rank * rows:(rank + 1) * rows].contiguous()
         v_loc = d["valid"][rank * rows:(rank + 1) * rows].contiguous()
         valid_tokens = int(d["valid"].sum().item())
@@ -533,7 +535,7 @@ def run_tp(args):
                 "timing": "eager TP forward per step (all_gather, layer, partial return, reduce)",
                 "config": {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens,
                            "rows_per_rank": rows, "H": w.H, "E": w.E, "k": w.k, "I": w.I,
-                           "S": w.S, "parallelism": f"tp{ws_n}",
+                           "S": w.S, "parallelism": f"{args.tp_layout}{ws_n}",
                            "partial_return": args.tp_return,
                            "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps"},
                 "clocks": clk}))
@@ -595,6 +597,9 @@ def main(argv=None):
     ap.add_argument("--tp", action="store_true",
                     help="tensor-parallel layout over the N ranks (default workload: dp_padded)")
     ap.add_argument("--tp-return", default="fused", choices=["fused", "nccl"])
+    ap.add_argument("--tp-layout", default="tp", choices=["tp", "ep"],
+                    help="with --tp: split every expert's intermediate dimension (tp) or "
+                         "the experts (ep) over the ranks")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the number of routed experts (profiling on a smaller case)")
     args = ap.parse_args(argv)

@@ -183,6 +183,25 @@ moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights *weights, cons
 moe_status moe_reduce_partials(const float *slots, int n_slots, int rows, int H,
                                const uint8_t *valid, void *out, void *stream);
 
+/* Expert-parallel rank: moe_forward_scatter restricted to the routed experts
+ * [expert_begin, expert_end) of the plan's num_experts.  Routing (logits, top-k,
+ * weights) is computed over all experts from the router weights as usual; pairs
+ * routed to other experts are left out of this rank's permutation (their groups
+ * stay empty and cost nothing) and out of its combine, so each token's fp32 sum
+ * is its share over this rank's experts (plus the shared expert's, when the
+ * plan has one: split its intermediate dimension over the ranks as in the
+ * tensor-parallel layout).  The routed weights given hold only these experts:
+ * w_gate_up [expert_end - expert_begin, 2I, H], w_down [.., H, I] and, for FP8,
+ * their scales; expert e's rows are at index e - expert_begin.  Summed over
+ * the ranks (moe_reduce_partials), the partials give the layer.  Requires
+ * 0 <= expert_begin < expert_end <= num_experts; other arguments as
+ * moe_forward_scatter, which is this call with the full range. */
+moe_status moe_forward_scatter_experts(moe_plan_t plan, const moe_weights *weights,
+                                       const void *hidden, const uint8_t *valid, int T, int k,
+                                       float *const *dst, int n_dst, int rows_per_rank, int slot,
+                                       int expert_begin, int expert_end, void *workspace,
+                                       size_t ws_bytes, void *stream, moe_debug *dbg);
+
 /* Routing only, from given fp32 logits [T, E] (device): the top-k selection,
  * weights, per-expert offsets and permutation exactly as moe_forward computes
  * them.  Outputs as in moe_debug (topk_ids, topk_w [T,k]; perm [T*k];

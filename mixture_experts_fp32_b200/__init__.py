@@ -32,7 +32,7 @@ MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")
 
 EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
-            "moe_forward_scatter", "moe_reduce_partials",
+            "moe_forward_scatter", "moe_forward_scatter_experts", "moe_reduce_partials",
             "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
             "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string")
 MAX_TP_RANKS = 8
@@ -98,6 +98,11 @@ def load():
                                       ctypes.POINTER(_vp), _c_int, _c_int, _c_int, _vp,
                                       ctypes.c_size_t, _vp, ctypes.POINTER(moe_debug)]
     L.moe_forward_scatter.restype = _c_int
+    L.moe_forward_scatter_experts.argtypes = [_vp, ctypes.POINTER(moe_weights), _vp, _vp, _c_int,
+                                              _c_int, ctypes.POINTER(_vp), _c_int, _c_int, _c_int,
+                                              _c_int, _c_int, _vp, ctypes.c_size_t, _vp,
+                                              ctypes.POINTER(moe_debug)]
+    L.moe_forward_scatter_experts.restype = _c_int
     L.moe_reduce_partials.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]
     L.moe_reduce_partials.restype = _c_int
     L.moe_route_from_logits.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp,
@@ -202,6 +207,19 @@ def moe_forward_scatter(plan, weights: moe_weights, hidden, valid, T: int, k: in
     _check(st, "moe_forward_scatter")
 
 
+def moe_forward_scatter_experts(plan, weights: moe_weights, hidden, valid, T: int, k: int, dst,
+                                rows_per_rank: int, slot: int, expert_begin: int, expert_end: int,
+                                workspace, ws_bytes: int, stream=None,
+                                dbg: moe_debug | None = None) -> None:
+    arr = (_vp * len(dst))(*[_addr(d) for d in dst])
+    st = load().moe_forward_scatter_experts(plan, ctypes.byref(weights), _addr(hidden),
+                                            _addr(valid), T, k, arr, len(dst), rows_per_rank,
+                                            slot, expert_begin, expert_end, _addr(workspace),
+                                            ws_bytes, _stream(stream),
+                                            None if dbg is None else ctypes.byref(dbg))
+    _check(st, "moe_forward_scatter_experts")
+
+
 def moe_reduce_partials(slots, n_slots: int, rows: int, H: int, valid, out, stream=None) -> None:
     st = load().moe_reduce_partials(_addr(slots), n_slots, rows, H, _addr(valid), _addr(out),
                                     _stream(stream))
@@ -264,6 +282,13 @@ class Plan:
                         rows_per_rank: int, slot: int, stream=None, dbg=None):
         moe_forward_scatter(self.handle, weights, hidden, valid, hidden.shape[0], k, dst,
                             rows_per_rank, slot, self.workspace, self.ws_bytes, stream, dbg)
+
+    def forward_scatter_experts(self, weights: moe_weights, hidden, valid, k: int, dst,
+                                rows_per_rank: int, slot: int, expert_begin: int,
+                                expert_end: int, stream=None, dbg=None):
+        moe_forward_scatter_experts(self.handle, weights, hidden, valid, hidden.shape[0], k, dst,
+                                    rows_per_rank, slot, expert_begin, expert_end,
+                                    self.workspace, self.ws_bytes, stream, dbg)
 
     def route_from_logits(self, logits, valid, k: int, topk_ids, topk_w, perm, offsets,
                           stream=None):

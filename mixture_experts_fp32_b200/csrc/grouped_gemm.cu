@@ -53,6 +53,7 @@ struct Cfg {
 struct KParams {
   const int* group_offsets;
   int E, G;
+  int e_base;       // the routed weights start at expert e_base
   int kb_routed, kb_shared;
   int rows_per_expert;
   int m_routed, m_shared;
@@ -173,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile ti = decode_tile(t, ts, go, p);
         const bool routed = ti.g < p.E;
         const CUtensorMap* am = routed ? &tmA : &tmAs;
-        const int arow = (routed ? ti.g * p.rows_per_expert : 0) + ti.m * BM;
+        const int arow = (routed ? (ti.g - p.e_base) * p.rows_per_expert : 0) + ti.m * BM;
         const int up = routed ? p.up_routed : p.up_shared;
         const uint32_t bytes = C::A_BYTES + ti.n_mma * BK * 2;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
@@ -353,7 +354,7 @@ cudaError_t prepare_grouped_gemm_kernels() {
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   CUtensorMap tmA, tmAs, tmB16, tmB32, tmB64;
-  const uint64_t rows_routed = (uint64_t)a.E * a.rows_per_expert;
+  const uint64_t rows_routed = (uint64_t)a.n_local * a.rows_per_expert;
   if (!make_map_bf16(&tmA, a.a_routed, a.K_routed, rows_routed, BM)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
     const uint64_t rows_shared = (uint64_t)a.m_tiles_shared * BM * (a.gated ? 2 : 1);
@@ -371,6 +372,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   p.group_offsets = a.group_offsets;
   p.E = a.E;
   p.G = a.G;
+  p.e_base = a.e_base;
   p.kb_routed = a.K_routed / BK;
   p.kb_shared = a.K_shared / BK;
   p.rows_per_expert = a.rows_per_expert;

@@ -122,6 +122,7 @@ __device__ __forceinline__ void promote16(float2 (&acc)[32], int base, const uin
 struct KParams8 {
   const int* group_offsets;
   int E, G;
+  int e_base;                     // the routed weights and scales start at expert e_base
   int kb_routed, kb_shared;
   int rows_per_expert;            // weight rows of one routed expert
   int ft_routed, ft_shared;       // feature tiles per group
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
         const bool routed = ti.g < p.E;
         const CUtensorMap* wm = routed ? &tmW : &tmWs;
-        const int wrow = (routed ? ti.g * p.rows_per_expert : 0) + ti.f0;
+        const int wrow = (routed ? (ti.g - p.e_base) * p.rows_per_expert : 0) + ti.f0;
         const int up = routed ? p.up_routed : p.up_shared;
         const int brow0 = wrow, brow1 = GATED ? wrow + up : wrow + 128;
         const int arow = ti.row0;
@@ -365,7 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       e.f0 = ti.f0;
       e.nfeat = ti.nfeat;
       e.k_blocks = ti.k_blocks;
-      const float* sw = routed ? p.sw_routed + (size_t)ti.g * (p.rows_per_expert / 128) * ti.k_blocks
+      const float* sw = routed ? p.sw_routed + (size_t)(ti.g - p.e_base) *
+                                                   (p.rows_per_expert / 128) * ti.k_blocks
                                : p.sw_shared;
       // weight scale rows: gated -> gate block and up block of f0; down -> block of this half
       const int up = routed ? p.up_routed : p.up_shared;
@@ -570,7 +572,7 @@ cudaError_t prepare_grouped_gemm_fp8_kernels() {
 cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st) {
   CUtensorMap tmA, tmW, tmWs;
   if (!make_map_u8(&tmA, a.b, a.K_ld, (uint64_t)a.R_cap)) return cudaErrorInvalidValue;
-  const uint64_t rows_routed = (uint64_t)a.E * a.rows_per_expert;
+  const uint64_t rows_routed = (uint64_t)a.n_local * a.rows_per_expert;
   if (!make_map_u8(&tmW, a.a_routed, a.K_routed, rows_routed)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
     const uint64_t rows_shared = a.gated ? (uint64_t)2 * a.up_shared : (uint64_t)a.feat_shared;
@@ -583,6 +585,7 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   p.group_offsets = a.group_offsets;
   p.E = a.E;
   p.G = a.G;
+  p.e_base = a.e_base;
   p.kb_routed = a.K_routed / BK;
   p.kb_shared = a.K_shared / BK;
   p.rows_per_expert = a.rows_per_expert;

@@ -184,11 +184,14 @@ MOE_EXPORT moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns
 }
 
 // The forward pass; `co` says where the combine writes (the bf16 output, or
-// fp32 tensor-parallel partial rows).  Argument checks common to both entry
-// points are here; each entry point checks its own output arguments first.
+// fp32 partial rows of a tensor- / expert-parallel rank), and [eb, ee) which
+// routed experts this call computes (their weights are the ones given).
+// Argument checks common to the entry points are here; each entry point checks
+// its own output arguments first.
 static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const void* hidden,
                                const uint8_t* valid, int T, int k, const moe::CombineOut& co,
-                               void* workspace, size_t ws_bytes, void* stream, moe_debug* dbg) {
+                               int eb, int ee, void* workspace, size_t ws_bytes, void* stream,
+                               moe_debug* dbg) {
   moe_status s = check_common(plan, T, k, workspace, ws_bytes);
   if (s != MOE_OK) return s;
   if (wts == nullptr) return MOE_ERR_INVALID_ARG;
@@ -244,8 +247,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
                                     logits, ids, w, st));
   if (s != MOE_OK) return s;
   record(dbg, 2, st);
-  s = check_launch(moe::launch_route(ids, valid, T, E, k, S, goff, perm, inv, rowtok, status,
-                                     at<int>(workspace, plan->off_rscratch), st));
+  s = check_launch(moe::launch_route(ids, valid, T, E, k, S, eb, ee, goff, perm, inv, rowtok,
+                                     status, at<int>(workspace, plan->off_rscratch), st));
   if (s != MOE_OK) return s;
   record(dbg, 3, st);
   const bool fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
@@ -270,6 +273,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     ga.d = h;
     ga.group_offsets = goff;
     ga.E = E;
+    ga.e_base = eb;
+    ga.n_local = ee - eb;
     ga.G = G;
     ga.K_routed = H;
     ga.K_shared = H;
@@ -323,6 +328,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     fa.sd = at<float>(workspace, plan->off_sh);
     fa.group_offsets = goff;
     fa.E = E;
+    fa.e_base = eb;
+    fa.n_local = ee - eb;
     fa.G = G;
     fa.K_routed = H;
     fa.K_shared = H;
@@ -395,14 +402,19 @@ MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const
   moe::CombineOut co;
   memset(&co, 0, sizeof(co));
   co.bf16 = static_cast<__nv_bfloat16*>(out);
-  return forward_impl(plan, wts, hidden, valid, T, k, co, workspace, ws_bytes, stream, dbg);
+  return forward_impl(plan, wts, hidden, valid, T, k, co, 0, plan->cfg.num_experts, workspace,
+                      ws_bytes, stream, dbg);
 }
 
-MOE_EXPORT moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights* wts,
-                                          const void* hidden, const uint8_t* valid, int T, int k,
-                                          float* const* dst, int n_dst, int rows_per_rank,
-                                          int slot, void* workspace, size_t ws_bytes,
-                                          void* stream, moe_debug* dbg) {
+MOE_EXPORT moe_status moe_forward_scatter_experts(moe_plan_t plan, const moe_weights* wts,
+                                                  const void* hidden, const uint8_t* valid, int T,
+                                                  int k, float* const* dst, int n_dst,
+                                                  int rows_per_rank, int slot, int expert_begin,
+                                                  int expert_end, void* workspace,
+                                                  size_t ws_bytes, void* stream, moe_debug* dbg) {
+  if (plan == nullptr || expert_begin < 0 || expert_end <= expert_begin ||
+      expert_end > plan->cfg.num_experts)
+    return MOE_ERR_INVALID_ARG;
   if (dst == nullptr || n_dst < 1 || n_dst > moe::kMaxTpRanks || rows_per_rank < 1 ||
       (long long)n_dst * rows_per_rank != T || slot < 0 || slot >= n_dst)
     return MOE_ERR_INVALID_ARG;
@@ -414,7 +426,19 @@ MOE_EXPORT moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights* wt
   }
   co.rows_per_rank = rows_per_rank;
   co.slot = slot;
-  return forward_impl(plan, wts, hidden, valid, T, k, co, workspace, ws_bytes, stream, dbg);
+  return forward_impl(plan, wts, hidden, valid, T, k, co, expert_begin, expert_end, workspace,
+                      ws_bytes, stream, dbg);
+}
+
+MOE_EXPORT moe_status moe_forward_scatter(moe_plan_t plan, const moe_weights* wts,
+                                          const void* hidden, const uint8_t* valid, int T, int k,
+                                          float* const* dst, int n_dst, int rows_per_rank,
+                                          int slot, void* workspace, size_t ws_bytes,
+                                          void* stream, moe_debug* dbg) {
+  if (plan == nullptr) return MOE_ERR_INVALID_ARG;
+  return moe_forward_scatter_experts(plan, wts, hidden, valid, T, k, dst, n_dst, rows_per_rank,
+                                     slot, 0, plan->cfg.num_experts, workspace, ws_bytes, stream,
+                                     dbg);
 }
 
 MOE_EXPORT moe_status moe_reduce_partials(const float* slots, int n_slots, int rows, int H,
@@ -449,7 +473,7 @@ MOE_EXPORT moe_status moe_route_from_logits(moe_plan_t plan, const float* logits
   s = check_launch(moe::launch_topk(logits, 1, nullptr, valid, T, E, k, c.renormalize,
                                     at<float>(workspace, plan->off_logits), topk_ids, topk_w, st));
   if (s != MOE_OK) return s;
-  s = check_launch(moe::launch_route(topk_ids, valid, T, E, k, S, goff, perm,
+  s = check_launch(moe::launch_route(topk_ids, valid, T, E, k, S, 0, E, goff, perm,
                                      at<int>(workspace, plan->off_inv),
                                      at<int>(workspace, plan->off_rowtok), status,
                                      at<int>(workspace, plan->off_rscratch), st));

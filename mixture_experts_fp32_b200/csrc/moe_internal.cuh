@@ -38,6 +38,7 @@ struct GroupedGemmArgs {
   void* d;                     // output rows [R_cap, ldd]: bf16 (gated) or fp32 (down)
   const int* group_offsets;    // [G + 1] on the device
   int E, G;                    // routed experts, total groups (E + S)
+  int e_base, n_local;         // a_routed holds experts [e_base, e_base + n_local) only
   int K_routed, K_shared, K_ld;
   int rows_per_expert;         // 2I (gated) or H (down)
   int m_tiles_routed, m_tiles_shared;   // output tiles of 128 weight rows per group
@@ -64,6 +65,7 @@ struct GroupedGemmFp8Args {
   float* sd;                   // gated: h scales [R_cap, ldd / 128]
   const int* group_offsets;
   int E, G;
+  int e_base, n_local;            // a_routed / sa_routed hold experts [e_base, +n_local) only
   int K_routed, K_shared, K_ld;
   int rows_per_expert;
   int feat_routed, feat_shared;   // output features of a group (gated: I, Is; down: H)
@@ -103,7 +105,7 @@ cudaError_t launch_topk(const float* partial, int splits, const float* bias, con
 // (parallel chunks); nullptr runs the single-block kernel.
 int route_scratch_ints(int max_tokens, int E);
 cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int k, int S,
-                         int* group_offsets, int* perm, int* inv, int* row_token,
+                         int eb, int ee, int* group_offsets, int* perm, int* inv, int* row_token,
                          unsigned int* status, int* scratch, cudaStream_t st);
 cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_token,
                                const int* total_rows, int R_cap, __nv_bfloat16* xp,

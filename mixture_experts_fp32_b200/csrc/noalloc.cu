@@ -75,7 +75,7 @@ MOE_EXPORT moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float
                        reinterpret_cast<float*>(scratch + off_logits), topk_ids, topk_w,
                        st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe::launch_route(topk_ids, valid, T, (int)E, k, (int)S, goff, perm,
+  if (moe::launch_route(topk_ids, valid, T, (int)E, k, (int)S, 0, (int)E, goff, perm,
                         reinterpret_cast<int*>(scratch + off_inv),
                         reinterpret_cast<int*>(scratch + off_rowtok), status, nullptr,
                         st) != cudaSuccess)

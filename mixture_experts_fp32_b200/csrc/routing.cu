@@ -29,9 +29,12 @@ namespace {
 
 constexpr int kChunk = 1024;
 
+// Pairs routed to experts outside [eb, ee) (the experts this call computes; all of
+// them, 0..E, unless a rank of an expert-parallel layer owns only a range) are left
+// out of the permutation: their groups stay empty and their inverse entries are -1.
 __device__ __forceinline__ void set_bits(uint32_t (*bits)[32], const int* ids, const uint8_t* valid,
-                                         int T, int E, int k, int t, int warp, int lane,
-                                         unsigned int* status) {
+                                         int T, int E, int k, int eb, int ee, int t, int warp,
+                                         int lane, unsigned int* status) {
   if (t < T && (valid == nullptr || valid[t])) {
     for (int j = 0; j < k; ++j) {
       const int e = ids[(size_t)t * k + j];
@@ -39,14 +42,14 @@ __device__ __forceinline__ void set_bits(uint32_t (*bits)[32], const int* ids, c
         atomicOr(status, MOE_DEV_BAD_EXPERT_ID);
         continue;
       }
-      atomicOr(&bits[e][warp], 1u << lane);
+      if (e >= eb && e < ee) atomicOr(&bits[e][warp], 1u << lane);
     }
   }
 }
 
 __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ ids,
                                                         const uint8_t* __restrict__ valid, int T,
-                                                        int E, int k, int S,
+                                                        int E, int k, int S, int eb, int ee,
                                                         int* __restrict__ group_offsets,
                                                         int* __restrict__ perm,
                                                         int* __restrict__ inv,
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
     for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
     __syncthreads();
     const int t = c * kChunk + tid;
-    set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+    set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, status);
     const bool ok = t < T && (valid == nullptr || valid[t]);
     const uint32_t vb = __ballot_sync(0xffffffffu, ok);
     if (lane == 0) wvalid[warp] = __popc(vb);
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
     for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
     __syncthreads();
     const int t = c * kChunk + tid;
-    set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+    set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, status);
     const bool ok = t < T && (valid == nullptr || valid[t]);
     const uint32_t vb = __ballot_sync(0xffffffffu, ok);
     if (lane == 0) wvalid[warp] = __popc(vb);
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
       if (ok) {
         for (int j = 0; j < k; ++j) {
           const int e = ids[(size_t)t * k + j];
-          if (e < 0 || e >= E) {
+          if (e < eb || e >= ee || e >= E) {
             inv[(size_t)t * ks + j] = -1;
             continue;
           }
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
 // Identical results to route_kernel.
 __global__ void __launch_bounds__(1024, 1) route_count_kernel(const int* __restrict__ ids,
                                                               const uint8_t* __restrict__ valid,
-                                                              int T, int E, int k,
+                                                              int T, int E, int k, int eb, int ee,
                                                               int* __restrict__ chunk_cnt,
                                                               int* __restrict__ chunk_valid,
                                                               unsigned int* status) {
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(1024, 1) route_count_kernel(const int* __restr
   for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
   __syncthreads();
   const int t = c * kChunk + tid;
-  set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+  set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, status);
   const uint32_t vb = __ballot_sync(0xffffffffu, t < T && (valid == nullptr || valid[t]));
   if (lane == 0) wvalid[warp] = __popc(vb);
   __syncthreads();
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(1024, 1) route_scan_kernel(const int* __restri
 
 __global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
     const int* __restrict__ ids, const uint8_t* __restrict__ valid, int T, int E, int k, int S,
-    const int* __restrict__ chunk_base, const int* __restrict__ vbase,
+    int eb, int ee, const int* __restrict__ chunk_base, const int* __restrict__ vbase,
     const int* __restrict__ group_offsets, int* __restrict__ perm, int* __restrict__ inv,
     int* __restrict__ row_token, unsigned int* status) {
   __shared__ uint32_t bits[kMaxExperts][32];
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
   for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
   __syncthreads();
   const int t = c * kChunk + tid;
-  set_bits(bits, ids, valid, T, E, k, t, warp, lane, status);
+  set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, status);
   const bool ok = t < T && (valid == nullptr || valid[t]);
   const uint32_t vb = __ballot_sync(0xffffffffu, ok);
   if (lane == 0) wvalid[warp] = __popc(vb);
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
   }
   for (int j = 0; j < k; ++j) {
     const int e = ids[(size_t)t * k + j];
-    if (e < 0 || e >= E) {
+    if (e < eb || e >= ee || e >= E) {
       inv[(size_t)t * ks + j] = -1;
       continue;
     }
@@ -357,17 +360,17 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
         const YT* yv = y + (size_t)v * 8;
 #define MOE_LD(J) \
   Vec8<YT> r##J;  \
-  if (J < ks) r##J = ld8(yv + (size_t)rows[J] * H);
+  if (J < ks && rows[J] >= 0) r##J = ld8(yv + (size_t)rows[J] * H);
         MOE_LD(0) MOE_LD(1) MOE_LD(2) MOE_LD(3) MOE_LD(4) MOE_LD(5) MOE_LD(6) MOE_LD(7) MOE_LD(8)
 #undef MOE_LD
 #define MOE_FMA(J)                                                                 \
-  if (J < k) {                                                                     \
+  if (J < k && rows[J] >= 0) {                                                     \
     _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] =                         \
         fmaf(wts[J], elem8(r##J, i), acc[i]);                                      \
   }
         MOE_FMA(0) MOE_FMA(1) MOE_FMA(2) MOE_FMA(3) MOE_FMA(4) MOE_FMA(5) MOE_FMA(6) MOE_FMA(7)
 #undef MOE_FMA
-        if (S) {                                       // the shared expert's row, slot k
+        if (S && rows[k] >= 0) {                       // the shared expert's row, slot k
           const Vec8<YT>& rs = k == 1 ? r1 : k == 2 ? r2 : k == 3 ? r3 : k == 4 ? r4
                              : k == 5 ? r5 : k == 6 ? r6 : k == 7 ? r7 : r8;
 #pragma unroll
@@ -490,20 +493,20 @@ int route_scratch_ints(int max_tokens, int E) {
 }
 
 cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int k, int S,
-                         int* group_offsets, int* perm, int* inv, int* row_token,
+                         int eb, int ee, int* group_offsets, int* perm, int* inv, int* row_token,
                          unsigned int* status, int* scratch, cudaStream_t st) {
   const int nchunks = (T + kChunk - 1) / kChunk;
   if (nchunks <= 1 || scratch == nullptr) {
-    route_kernel<<<1, 1024, 0, st>>>(ids, valid, T, E, k, S, group_offsets, perm, inv, row_token,
-                                     status);
+    route_kernel<<<1, 1024, 0, st>>>(ids, valid, T, E, k, S, eb, ee, group_offsets, perm, inv,
+                                     row_token, status);
     return cudaGetLastError();
   }
   int* chunk_cnt = scratch;                        // [nchunks][E]
   int* chunk_base = chunk_cnt + (size_t)nchunks * E;   // [nchunks][E]
   int* chunk_valid = chunk_base + (size_t)nchunks * E; // [nchunks]
   int* vbase = chunk_valid + nchunks;                  // [nchunks]
-  route_count_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, chunk_cnt, chunk_valid,
-                                               status);
+  route_count_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, eb, ee, chunk_cnt,
+                                               chunk_valid, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   route_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, chunk_valid, nchunks, E, S, chunk_base, vbase,
@@ -511,8 +514,9 @@ cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // set_bits reports a bad expert id once in the count pass; the scatter pass skips it quietly
-  route_scatter_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, S, chunk_base, vbase,
-                                                 group_offsets, perm, inv, row_token, status);
+  route_scatter_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, S, eb, ee, chunk_base,
+                                                 vbase, group_offsets, perm, inv, row_token,
+                                                 status);
   return cudaGetLastError();
 }
 

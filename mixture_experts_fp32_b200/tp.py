@@ -24,6 +24,15 @@ local rows are split in two; the all_gather of the second runs on a communicatio
 while the first computes, and (nccl form) the first's reduce_scatter runs while the
 second computes.
 
+Expert parallelism uses the same gather and the same return: rank r owns the routed
+experts [r E/n, (r+1) E/n) (and 1/n of the shared expert's intermediate dimension);
+routing is still computed over all experts, pairs routed elsewhere are left out of its
+permutation (`moe_forward_scatter_experts`), and its combine returns each token's sum
+over its own experts.  The all_gather stands in for the dispatch and the fused partial
+return for the combine's all-to-all, so no kernel waits on another (the down GEMM's
+per-expert completion signals of an all-to-all combine are not needed: the return rides
+in the layer's last kernel).
+
 Row ownership: gathered row t belongs to rank t // rows, local row t % rows.
 """
 from __future__ import annotations
@@ -56,16 +65,48 @@ def shard_weights(full: Dict[str, Optional[torch.Tensor]], n: int, r: int, *, I:
         sgu = full["s_gate_up"]
         out["s_gate_up"] = torch.cat([sgu[:, b0:b1], sgu[:, bI + b0:bI + b1]], dim=1).contiguous()
         out["s_down"] = full["s_down"][:, :, b0:b1].contiguous()
-    if full.get("ws_gate_up") is not None:
-        j0, j1 = r * Is // n, (r + 1) * Is // n
-        ws = full["ws_gate_up"]
-        out["ws_gate_up"] = torch.cat([ws[j0:j1], ws[Is + j0:Is + j1]], dim=0).contiguous()
-        out["ws_down"] = full["ws_down"][:, j0:j1].contiguous()
-        if fp8:
-            c0, c1, cI = j0 // 128, j1 // 128, Is // 128
-            ss = full["ss_gate_up"]
-            out["ss_gate_up"] = torch.cat([ss[c0:c1], ss[cI + c0:cI + c1]], dim=0).contiguous()
-            out["ss_down"] = full["ss_down"][:, c0:c1].contiguous()
+    out.update(_shard_shared(full, n, r, Is=Is, fp8=fp8))
+    return out
+
+
+def _shard_shared(full, n: int, r: int, *, Is: int, fp8: bool) -> dict:
+    """1/n of the shared expert's intermediate dimension (empty dict without one)."""
+    out = {}
+    if full.get("ws_gate_up") is None:
+        return out
+    if Is % (128 * n):
+        raise ValueError("each rank's share of the shared expert must be a multiple of 128")
+    j0, j1 = r * Is // n, (r + 1) * Is // n
+    ws = full["ws_gate_up"]
+    out["ws_gate_up"] = torch.cat([ws[j0:j1], ws[Is + j0:Is + j1]], dim=0).contiguous()
+    out["ws_down"] = full["ws_down"][:, j0:j1].contiguous()
+    if fp8:
+        c0, c1, cI = j0 // 128, j1 // 128, Is // 128
+        ss = full["ss_gate_up"]
+        out["ss_gate_up"] = torch.cat([ss[c0:c1], ss[cI + c0:cI + c1]], dim=0).contiguous()
+        out["ss_down"] = full["ss_down"][:, c0:c1].contiguous()
+    return out
+
+
+def expert_range(E: int, n: int, r: int):
+    """The routed experts rank r owns in the expert-parallel layout."""
+    if E % n:
+        raise ValueError("the routed experts must divide by the number of ranks")
+    return r * E // n, (r + 1) * E // n
+
+
+def shard_experts(full: Dict[str, Optional[torch.Tensor]], n: int, r: int, *, E: int, Is: int,
+                  fp8: bool) -> Dict[str, Optional[torch.Tensor]]:
+    """Rank r's share in the expert-parallel layout: its routed experts whole, and 1/n
+    of the shared expert's intermediate dimension (as in the tensor-parallel shard)."""
+    e0, e1 = expert_range(E, n, r)
+    out = {"router_w": full["router_w"], "router_b": full.get("router_b")}
+    out["w_gate_up"] = full["w_gate_up"][e0:e1].contiguous()
+    out["w_down"] = full["w_down"][e0:e1].contiguous()
+    if fp8:
+        out["s_gate_up"] = full["s_gate_up"][e0:e1].contiguous()
+        out["s_down"] = full["s_down"][e0:e1].contiguous()
+    out.update(_shard_shared(full, n, r, Is=Is, fp8=fp8))
     return out
 
 
@@ -87,13 +128,14 @@ def split_rows(rows: int):
 
 
 class TPMoE:
-    """One rank of the tensor-parallel layer.  `full` holds the whole layer's weights on
-    this rank's device (the shard is cut from it); `rows` is the number of rows each
-    DP rank contributes per micro-batch (padding rows included, marked invalid)."""
+    """One rank of the tensor-parallel layer (layout "tp") or of the expert-parallel one
+    (layout "ep").  `full` holds the whole layer's weights on this rank's device (the
+    shard is cut from it); `rows` is the number of rows each DP rank contributes per
+    micro-batch (padding rows included, marked invalid)."""
 
     def __init__(self, full: dict, *, E: int, H: int, I: int, S: int, Is: int, k_max: int,
                  rows: int, fp8: bool = False, fused: bool = True, group=None,
-                 barrier_timeout_ms: int = 10000):
+                 barrier_timeout_ms: int = 10000, layout: str = "tp"):
         import torch.distributed as dist
         self.group = group if group is not None else dist.group.WORLD
         self.n = dist.get_world_size(group)
@@ -102,12 +144,19 @@ class TPMoE:
             raise ValueError("at most 8 tensor-parallel ranks")
         self.H, self.rows, self.fused = H, rows, fused
         self.timeout_ms = barrier_timeout_ms
-        self.shard = shard_weights(full, self.n, self.rank, I=I, Is=Is, fp8=fp8)
+        if layout == "tp":
+            self.shard = shard_weights(full, self.n, self.rank, I=I, Is=Is, fp8=fp8)
+            self.experts, inter = (0, E), I // self.n
+        elif layout == "ep":
+            self.shard = shard_experts(full, self.n, self.rank, E=E, Is=Is, fp8=fp8)
+            self.experts, inter = expert_range(E, self.n, self.rank), I
+        else:
+            raise ValueError(layout)
         self.weights = make_shard_weights(self.shard)
         dev = full["w_gate_up"].device
         T = self.n * rows
         self.plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
-                             inter=I // self.n, num_shared=S, shared_inter=Is // self.n if S else 0,
+                             inter=inter, num_shared=S, shared_inter=Is // self.n if S else 0,
                              wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16, device=dev)
         self.x_all = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.valid_all = torch.empty(T, dtype=torch.uint8, device=dev)
@@ -135,14 +184,16 @@ class TPMoE:
         import torch.distributed as dist
         if self.fused:
             par = self.step & 1
-            self.plan.forward_scatter(self.weights, self.x_all, self.valid_all, k, self.dst[par],
-                                      self.rows, self.rank)
+            self.plan.forward_scatter_experts(self.weights, self.x_all, self.valid_all, k,
+                                              self.dst[par], self.rows, self.rank,
+                                              *self.experts)
             self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
             moe.moe_reduce_partials(self.slab[par], self.n, self.rows, self.H, valid_local,
                                     out_local)
         else:
-            self.plan.forward_scatter(self.weights, self.x_all, self.valid_all, k,
-                                      [self.partial], self.n * self.rows, 0)
+            self.plan.forward_scatter_experts(self.weights, self.x_all, self.valid_all, k,
+                                              [self.partial], self.n * self.rows, 0,
+                                              *self.experts)
             dist.reduce_scatter_tensor(self.recv, self.partial, op=dist.ReduceOp.SUM,
                                        group=self.group)
             moe.moe_reduce_partials(self.recv, 1, self.rows, self.H, valid_local, out_local)
@@ -182,9 +233,10 @@ class TPMoETwoBatch:
 
 
 def tp_forward_reference(full: dict, x_rows: List[torch.Tensor], valid_rows: List[torch.Tensor],
-                         k: int, *, E, H, I, S, Is, k_max, fp8, n_shards: int):
-    """One-GPU emulation of n ranks (no process group): every shard's forward scatters
-    into every owner's slab, then each owner reduces.  Returns the owners' outputs."""
+                         k: int, *, E, H, I, S, Is, k_max, fp8, n_shards: int, layout: str = "tp"):
+    """One-GPU emulation of n ranks (no process group) of either layout: every rank's
+    forward scatters into every owner's slab, then each owner reduces.  Returns the
+    owners' outputs."""
     dev = full["w_gate_up"].device
     rows = x_rows[0].shape[0]
     x_all = torch.cat(x_rows)
@@ -194,13 +246,17 @@ def tp_forward_reference(full: dict, x_rows: List[torch.Tensor], valid_rows: Lis
              for _ in range(n_shards)]
     plans = []
     for r in range(n_shards):
-        sh = shard_weights(full, n_shards, r, I=I, Is=Is, fp8=fp8)
+        if layout == "tp":
+            sh = shard_weights(full, n_shards, r, I=I, Is=Is, fp8=fp8)
+            experts, inter = (0, E), I // n_shards
+        else:
+            sh = shard_experts(full, n_shards, r, E=E, Is=Is, fp8=fp8)
+            experts, inter = expert_range(E, n_shards, r), I
         plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
-                        inter=I // n_shards, num_shared=S,
-                        shared_inter=Is // n_shards if S else 0,
+                        inter=inter, num_shared=S, shared_inter=Is // n_shards if S else 0,
                         wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16, device=dev)
-        plan.forward_scatter(make_shard_weights(sh), x_all, v_all, k, [s for s in slabs],
-                             rows, r)
+        plan.forward_scatter_experts(make_shard_weights(sh), x_all, v_all, k, [s for s in slabs],
+                                     rows, r, *experts)
         plans.append((plan, sh))
     outs = []
     for r in range(n_shards):

@@ -1,13 +1,15 @@
-"""The tensor-parallel layer on one GPU.
+"""The tensor- and expert-parallel layers on one GPU.
 
 * n shards emulated in one process: every shard's forward scatters its fp32 partial rows
   into every owner's slab, each owner sums its slab in rank order and rounds once; the
   owners' outputs must match the oracle's whole layer (same tolerance as the layer) and
   the unsharded forward, and padding rows must be +0.0.
+* the same for the expert-parallel layout: each rank computes its own experts (pairs
+  routed elsewhere left out of its permutation and combine) and 1/n of the shared expert;
 * a one-rank NCCL process group runs the TPMoE class (fused path through symmetric
-  memory, and the NCCL reduce_scatter path) and the two-micro-batch schedule; with one
-  rank the shard is the whole layer, so each must give the unsharded forward's output
-  bit for bit."""
+  memory, and the NCCL reduce_scatter path, both layouts) and the two-micro-batch
+  schedule; with one rank the shard is the whole layer, so each must give the unsharded
+  forward's output bit for bit."""
 import os
 import socket
 
@@ -35,16 +37,25 @@ def built():
 
 CASES = [
     (Workload("tp2_bf16_padded", T=4 * 48, H=512, E=16, k=3, I=512, S=1, Is=256,
-              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 2),
+              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 2, "tp"),
     (Workload("tp4_bf16_padded", T=4 * 48, H=512, E=16, k=3, I=512, S=1, Is=512,
-              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 4),
+              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 4, "tp"),
     (Workload("tp2_fp8", T=2 * 64, H=512, E=8, k=2, I=256, S=1, Is=256, wtype="fp8",
-              router_sigma=0.2, w_sigma=0.05), 2),
+              router_sigma=0.2, w_sigma=0.05), 2, "tp"),
+    (Workload("ep2_bf16_padded", T=4 * 48, H=512, E=16, k=3, I=256, S=1, Is=256,
+              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 2, "ep"),
+    (Workload("ep4_bf16_zipf", T=4 * 64, H=512, E=16, k=4, I=256, S=1, Is=512,
+              router_sigma=0.2, bias="zipf"), 4, "ep"),
+    (Workload("ep2_fp8", T=2 * 64, H=512, E=8, k=2, I=256, S=1, Is=256, wtype="fp8",
+              router_sigma=0.2, w_sigma=0.05), 2, "ep"),
+    (Workload("ep4_fp8_no_shared", T=4 * 32, H=512, E=8, k=3, I=256, S=0, Is=0, wtype="fp8",
+              router_sigma=0.2, w_sigma=0.05), 4, "ep"),
 ]
 
 
-@pytest.mark.parametrize("w,n", CASES, ids=lambda c: c.name if hasattr(c, "name") else str(c))
-def test_emulated_ranks_match_the_layer(w, n):
+@pytest.mark.parametrize("w,n,layout", CASES,
+                         ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_emulated_ranks_match_the_layer(w, n, layout):
     inp = synth.make_inputs(w)
     d = to_device(inp)
     rows = w.T // n
@@ -52,7 +63,7 @@ def test_emulated_ranks_match_the_layer(w, n):
     xs = [d["x"][r * rows:(r + 1) * rows] for r in range(n)]
     vs = [d["valid"][r * rows:(r + 1) * rows] for r in range(n)]
     outs = tp.tp_forward_reference(d, xs, vs, w.k, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is,
-                                   k_max=w.k, fp8=w.wtype == "fp8", n_shards=n)
+                                   k_max=w.k, fp8=w.wtype == "fp8", n_shards=n, layout=layout)
     got = torch.cat(outs).cpu()
     res = dict(full_res)
     res["out"] = got
@@ -82,14 +93,15 @@ def one_rank_group():
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("fused", [True, False], ids=["fused", "nccl"])
-def test_one_rank_tp_equals_the_layer(one_rank_group, fused):
+@pytest.mark.parametrize("fused,layout", [(True, "tp"), (False, "tp"), (True, "ep")],
+                         ids=["tp-fused", "tp-nccl", "ep-fused"])
+def test_one_rank_tp_equals_the_layer(one_rank_group, fused, layout):
     w = Workload("tp1", T=64, H=512, E=16, k=3, I=512, S=1, Is=256, router_sigma=0.2,
                  mask="dp_padded", dp_rows=(40,))
     d = to_device(synth.make_inputs(w))
     ref = run_forward(plan_for(w), d, w.k)["out"]
     layer = tp.TPMoE(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is, k_max=w.k, rows=w.T,
-                     fp8=False, fused=fused)
+                     fp8=False, fused=fused, layout=layout)
     for _ in range(3):                                   # alternate slabs across steps
         out = torch.full((w.T, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
         layer.forward(d["x"], d["valid"], w.k, out)

@@ -90,3 +90,31 @@ def test_shard_rejects_uneven_splits():
         tp.shard_weights(inp, 3, 0, I=w.I, Is=w.Is, fp8=False)
     with pytest.raises(ValueError):
         tp.shard_weights(inp, 4, 0, I=w.I, Is=w.Is, fp8=True)   # 64-wide shard
+
+
+@pytest.mark.parametrize("w", [
+    Workload("ep_bf16", T=24, H=256, E=8, k=3, I=256, S=1, Is=512, router_sigma=0.2),
+    Workload("ep_fp8", T=24, H=256, E=8, k=3, I=256, S=1, Is=256, wtype="fp8",
+             router_sigma=0.2, w_sigma=0.05),
+], ids=lambda w: w.name)
+def test_expert_shards_sum_to_the_layer(w):
+    """Expert-parallel layout: each rank's routed experts whole (pairs routed elsewhere
+    contribute nothing there) plus 1/n of the shared expert; the ranks' accumulators,
+    from the oracle on each rank's own weights, sum to the layer's."""
+    inp = synth.make_inputs(w)
+    fp8 = w.wtype == "fp8"
+    full = oracle.forward(inp)
+    ids, wts = full["ids"], full["w"]
+    for n in (2, 4) if not fp8 else (2,):
+        acc = np.zeros_like(full["acc"])
+        for r in range(n):
+            e0, e1 = tp.expert_range(w.E, n, r)
+            sh = tp.shard_experts(inp, n, r, E=w.E, Is=w.Is, fp8=fp8)
+            local = (ids >= e0) & (ids < e1)
+            rank_inp = dict(inp)
+            rank_inp.update(sh)
+            rank_inp["workload"] = w.with_(E=e1 - e0, Is=w.Is // n)
+            acc += oracle.moe_tokens(rank_inp, np.where(local, ids - e0, 0).astype(np.int32),
+                                     np.where(local, wts, 0.0))
+        assert np.abs(acc - full["acc"]).max() <= 1e-12 * np.abs(full["acc"]).max()
+        assert tp.expert_range(w.E, n, n - 1)[1] == w.E
