@@ -31,7 +31,7 @@ L2_FLUSH_BYTES = 512 << 20
 # DRAM traffic / algorithmic bytes of one gate/up GEMM launch, from the ncu capture
 # summarised in profiles/grouped_gemm_step3_e8.md; it applies only to the kernel
 # source it was measured on (sha256 prefix), and "traffic" is null otherwise.
-GEMM_TRAFFIC = {"sha256_prefix": "82080a022417b183", "gate_up_ratio": 0.997}
+GEMM_TRAFFIC = {"sha256_prefix": "0ed45de09043589f", "gate_up_ratio": 0.998}
 
 
 def gemm_source_hash() -> str:

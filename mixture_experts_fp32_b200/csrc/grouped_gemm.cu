@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmAs,
                         const __grid_constant__ CUtensorMap tmB16,
                         const __grid_constant__ CUtensorMap tmB32,
-                        const __grid_constant__ CUtensorMap tmB64, const KParams p) {
+                        const __grid_constant__ CUtensorMap tmB64,
+                        const __grid_constant__ CUtensorMap tmB128, const KParams p) {
   using C = Cfg<GATED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB16);
     tma_prefetch_desc(&tmB32);
     tma_prefetch_desc(&tmB64);
+    tma_prefetch_desc(&tmB128);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
@@ -176,7 +178,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* am = routed ? &tmA : &tmAs;
         const int arow = (routed ? (ti.g - p.e_base) * p.rows_per_expert : 0) + ti.m * BM;
         const int up = routed ? p.up_routed : p.up_shared;
-        const uint32_t bytes = C::A_BYTES + ti.n_mma * BK * 2;
+        // the tile's rows in one box of 16/32/64/128 rows (one copy from the single
+        // producer thread per K block; rows past the group come from L2 and go unused)
+        const int box = ti.n_mma <= 16 ? 16 : ti.n_mma <= 32 ? 32 : ti.n_mma <= 64 ? 64 : 128;
+        const CUtensorMap* bm =
+            box == 16 ? &tmB16 : box == 32 ? &tmB32 : box == 64 ? &tmB64 : &tmB128;
+        const uint32_t bytes = C::A_BYTES + box * BK * 2;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, p.wait_limit_ns, p.status,
                                  p.timeout_bit)) {
@@ -189,15 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(a_dst, am, kb * BK, arow, fb, pol_a);
           if (GATED) tma_load_2d(a_dst + BM * BK * 2, am, kb * BK, arow + up, fb, pol_a);
           const uint32_t b_dst = smem_u32(b_smem + stage * C::B_BYTES);
-          // the tile's rows in at most three boxes (64 / 32 / 16 rows): one thread
-          // issues every copy, and a copy per 16 rows left it behind the weight stream
-          for (int r = 0; r < ti.n_mma;) {
-            const int left = ti.n_mma - r;
-            const int box = left >= 64 ? 64 : left >= 32 ? 32 : 16;
-            const CUtensorMap* bm = box == 64 ? &tmB64 : box == 32 ? &tmB32 : &tmB16;
-            tma_load_2d(b_dst + r * BK * 2, bm, kb * BK, ti.row0 + r, fb, pol_b);
-            r += box;
-          }
+          tma_load_2d(b_dst, bm, kb * BK, ti.row0, fb, pol_b);
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -353,7 +352,7 @@ cudaError_t prepare_grouped_gemm_kernels() {
 }
 
 cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
-  CUtensorMap tmA, tmAs, tmB16, tmB32, tmB64;
+  CUtensorMap tmA, tmAs, tmB16, tmB32, tmB64, tmB128;
   const uint64_t rows_routed = (uint64_t)a.n_local * a.rows_per_expert;
   if (!make_map_bf16(&tmA, a.a_routed, a.K_routed, rows_routed, BM)) return cudaErrorInvalidValue;
   if (a.a_shared != nullptr) {
@@ -365,7 +364,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   }
   if (!make_map_bf16(&tmB16, a.b, a.K_ld, (uint64_t)a.R_cap, 16) ||
       !make_map_bf16(&tmB32, a.b, a.K_ld, (uint64_t)a.R_cap, 32) ||
-      !make_map_bf16(&tmB64, a.b, a.K_ld, (uint64_t)a.R_cap, 64))
+      !make_map_bf16(&tmB64, a.b, a.K_ld, (uint64_t)a.R_cap, 64) ||
+      !make_map_bf16(&tmB128, a.b, a.K_ld, (uint64_t)a.R_cap, 128))
     return cudaErrorInvalidValue;
 
   KParams p;
@@ -387,10 +387,10 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   p.wait_limit_ns = a.wait_limit_ns;
   if (a.gated) {
     grouped_gemm_kernel<true><<<a.num_ctas, kThreads, Cfg<true>::SMEM_BYTES, st>>>(
-        tmA, tmAs, tmB16, tmB32, tmB64, p);
+        tmA, tmAs, tmB16, tmB32, tmB64, tmB128, p);
   } else {
     grouped_gemm_kernel<false><<<a.num_ctas, kThreads, Cfg<false>::SMEM_BYTES, st>>>(
-        tmA, tmAs, tmB16, tmB32, tmB64, p);
+        tmA, tmAs, tmB16, tmB32, tmB64, tmB128, p);
   }
   return cudaGetLastError();
 }
