@@ -136,13 +136,10 @@ __global__ void __launch_bounds__(RThreads, 1)
       const uint32_t idesc = idesc_bf16_m128(n);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_sleep(smem_u32(&full[stage]), phase, kRouterWaitNs, p.status,
-                             p.timeout_bit)) {
-          ok = false;
-          break;
-        }
+                             p.timeout_bit))
+          break;   // status bit set; commit below still drains what was issued
         tc_fence_after();
         const uint64_t a_desc = smem_desc_sw128(smem_u32(a_smem + stage * RA_BYTES));
 #pragma unroll
@@ -162,7 +159,6 @@ __global__ void __launch_bounds__(RThreads, 1)
       // tensor memory is released
       umma_commit(smem_u32(tfull));
       mbar_wait_sleep(smem_u32(tfull), 0, kRouterWaitNs, p.status, p.timeout_bit);
-      (void)ok;
     }
     __syncwarp();
   } else {
