@@ -159,3 +159,19 @@ def test_tensor_parallel_entry_points_reject_bad_arguments_before_launch(lib):
         assert red(0x7000, 2, 0, 64, None, 0x9000, None) == moe.MOE_OK                 # no rows
     finally:
         moe.moe_plan_destroy(plan)
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """The header compiles as C99 and a C program linked to the library gets the
+    documented host-side behaviour (no GPU involved)."""
+    exe = tmp_path / "host_only"
+    libdir = os.path.dirname(moe.LIB_PATH)
+    libname = os.path.basename(moe.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c", "host_only.c"),
+                           "-o", str(exe), "-L", libdir, "-l:" + libname,
+                           "-Wl,-rpath," + libdir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr + out.stdout
+    assert "passed" in out.stdout
