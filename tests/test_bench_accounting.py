@@ -1,0 +1,54 @@
+"""The benchmark's roofline accounting against the step budgets worked out by hand for
+each workload with every routed expert touched (bytes the layer must move: touched
+experts' and the shared expert's weights, the router, valid input rows, all output rows;
+flops of the expert FFNs and of the router)."""
+import numpy as np
+import pytest
+
+import bench
+import synth
+
+# (workload, step GB, expert GFLOP, router GFLOP), all experts touched
+BUDGETS = [
+    ("step3_decode", 10.80, 225.5, 0.18),
+    ("deepseek_decode", 22.65, 101.5, 0.47),
+    ("dp_padded", 10.70, 750.4, 0.78),
+    ("fp8_prefill", 11.56, 6494.0, 30.1),
+]
+
+
+@pytest.mark.parametrize("name,gb,gflop,router_gflop", BUDGETS)
+def test_step_budget(name, gb, gflop, router_gflop):
+    w = synth.WORKLOADS[name]
+    valid = int(synth.workloads.valid_mask(w).sum())
+    pairs = valid * w.k
+    counts = np.full(w.E, pairs // w.E)
+    counts[: pairs - counts.sum()] += 1              # every expert touched
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    a = bench.algorithmic(w, valid, offsets, w.k)
+    assert a["touched_experts"] == w.E and a["routed_rows"] == pairs
+    assert abs(a["step_bytes"] / 1e9 - gb) <= 0.006 * gb
+    assert abs(a["expert_flops"] / 1e9 - gflop) <= 0.002 * gflop
+    assert abs((a["step_flops"] - a["expert_flops"]) / 1e9 - router_gflop) <= 0.03 * router_gflop + 0.01
+    # the gate/up kernel's share: two of the three expert matmuls
+    assert abs(a["gate_up_flops"] / a["expert_flops"] - 2 / 3) < 1e-12
+
+
+def test_untouched_experts_cost_no_weight_bytes():
+    w = synth.WORKLOADS["step3_decode"]
+    full = bench.algorithmic(w, w.T, np.arange(0, 49 * 16, 16), w.k)
+    counts = np.zeros(w.E, dtype=int)
+    counts[:10] = w.T * w.k // 10
+    counts[0] += w.T * w.k - counts.sum()
+    part = bench.algorithmic(w, w.T, np.concatenate([[0], np.cumsum(counts)]), w.k)
+    per_expert = 3 * w.H * w.I * 2                   # gate, up and down, bf16
+    assert part["touched_experts"] == 10
+    assert full["step_bytes"] - part["step_bytes"] == (w.E - 10) * per_expert
+
+
+def test_launch_count_per_step():
+    # weight split, router, top-k; the permutation (1 kernel up to 1024 rows, 3 above);
+    # the gather or FP8 quantisation; two GEMMs; the combine. The decode figure is the
+    # eight kernels a launch list of one decode step shows.
+    assert bench.launches_per_step(synth.WORKLOADS["step3_decode"]) == 8
+    assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 10
