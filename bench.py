@@ -65,6 +65,15 @@ def launches_per_step(w) -> int:
     return 3 + route + 1 + 2 + 1
 
 
+def step_spread(ms) -> dict:
+    """Median and 10th / 90th percentiles (linear interpolation) of per-step times."""
+    import numpy as np
+    if not ms:
+        return {"p10": None, "p50": None, "p90": None}
+    q = np.percentile(np.asarray(ms, dtype=np.float64), [10, 50, 90])
+    return {"p10": float(q[0]), "p50": float(q[1]), "p90": float(q[2])}
+
+
 def replica_seed(seed: int, rank: int) -> int:
     """Seed of a replica's own batch of hidden states (rank 0 keeps the workload's)."""
     return seed + 1000 * rank
@@ -387,13 +396,23 @@ def run_native(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes": algo["gate_up_bytes"],
                          "algorithmic_flops": algo["gate_up_flops"],
-                         "launch_ms": gemm_ms, "peak_source": peaks["source"]},
+                         "launch_ms": gemm_ms, "peak_source": peaks["source"],
+                         # the same kernel against the matmul rate measured over seconds
+                         # under the power cap (the timed steps run back to back)
+                         "frac_of_sustained": (achieved / (peaks["bf16_tflops_sustained"]
+                                                           * (2 if w.wtype == "fp8" else 1))
+                                               if bound == "tensor"
+                                               and peaks.get("bf16_tflops_sustained")
+                                               else None)},
             "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / head_ms,
                               "frac_eager": step_roof_ms / ms,
                               "algorithmic_bytes": algo["step_bytes"],
                               "algorithmic_flops": algo["step_flops"],
                               "touched_experts": algo["touched_experts"]},
             "stage_ms": stage_ms,
+            "step_ms_spread": {"rank": 0, "eager": step_spread(step_ms),
+                               "graph": step_spread(gms) if graph_ms is not None else None,
+                               "e2e": step_spread(e2e_ms)},
             "e2e": {"value": tokens / (e2e_total * 1e-3 / K), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_host.numel() * 2 + v_host.numel(),
                     "d2h_bytes_per_step": out_host.numel() * 2},

@@ -52,3 +52,9 @@ def test_launch_count_per_step():
     # eight kernels a launch list of one decode step shows.
     assert bench.launches_per_step(synth.WORKLOADS["step3_decode"]) == 8
     assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 10
+
+
+def test_step_spread():
+    s = bench.step_spread([float(v) for v in range(1, 12)])     # 1..11 ms
+    assert s == {"p10": 2.0, "p50": 6.0, "p90": 10.0}
+    assert bench.step_spread([]) == {"p10": None, "p50": None, "p90": None}
