@@ -227,9 +227,9 @@ def run_native(args):
     plan = moe.Plan(max_tokens=w.T, hidden=w.H, num_experts=w.E, top_k_max=k, inter=w.I,
                     num_shared=w.S, shared_inter=w.Is if w.S else 0, device=dev,
                     wtype=moe.MOE_W_BF16 if w.wtype == "bf16" else moe.MOE_W_FP8_E4M3_B128)
-    weights = moe.make_weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
-                               d.get("s_gate_up"), d.get("s_down"), d.get("ws_gate_up"),
-                               d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
+    weights = plan.weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
+                           d.get("s_gate_up"), d.get("s_down"), d.get("ws_gate_up"),
+                           d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
     out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
     offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)

@@ -123,12 +123,31 @@ def load():
     return L
 
 
-def _addr(t) -> int | None:
-    """Device (or host) address of a tensor, an int address, or None."""
+# element types accepted for each kind of tensor argument (torch dtype names)
+_F32 = ("float32",)
+_I32 = ("int32",)
+_BF16 = ("bfloat16",)
+_MASK = ("uint8", "bool")
+_WEIGHT = ("bfloat16", "uint8", "float8_e4m3fn")
+
+
+def _addr(t, name: str = "argument", dtypes=None) -> int | None:
+    """Address of a tensor argument, or an int taken as a raw address, or None.
+
+    A tensor must be a contiguous CUDA tensor (of one of ``dtypes`` when given):
+    the kernels read and write it as a dense row-major array in device memory, so a
+    host tensor, a strided view or a wrong element type is refused here, before
+    anything is enqueued, instead of being read out of bounds on the device."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError(f"{name}: a CUDA tensor is required, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: a contiguous tensor is required")
+    if dtypes is not None and str(t.dtype).rsplit(".", 1)[-1] not in dtypes:
+        raise ValueError(f"{name}: element type {t.dtype} is not one of {', '.join(dtypes)}")
     return t.data_ptr()
 
 
@@ -174,13 +193,18 @@ def moe_plan_set_wait_limit(plan, limit_ns: int) -> None:
 def make_weights(router_w, router_b=None, w_gate_up=None, w_down=None, s_gate_up=None,
                  s_down=None, ws_gate_up=None, ws_down=None, ss_gate_up=None,
                  ss_down=None) -> moe_weights:
-    return moe_weights(*[_addr(t) for t in (router_w, router_b, w_gate_up, w_down, s_gate_up,
-                                             s_down, ws_gate_up, ws_down, ss_gate_up, ss_down)])
+    return moe_weights(_addr(router_w, "router_w", _F32), _addr(router_b, "router_b", _F32),
+                       _addr(w_gate_up, "w_gate_up", _WEIGHT), _addr(w_down, "w_down", _WEIGHT),
+                       _addr(s_gate_up, "s_gate_up", _F32), _addr(s_down, "s_down", _F32),
+                       _addr(ws_gate_up, "ws_gate_up", _WEIGHT), _addr(ws_down, "ws_down", _WEIGHT),
+                       _addr(ss_gate_up, "ss_gate_up", _F32), _addr(ss_down, "ss_down", _F32))
 
 
 def make_debug(logits=None, topk_ids=None, topk_w=None, perm=None, offsets=None,
                events=None) -> moe_debug:
-    d = moe_debug(_addr(logits), _addr(topk_ids), _addr(topk_w), _addr(perm), _addr(offsets))
+    d = moe_debug(_addr(logits, "logits", _F32), _addr(topk_ids, "topk_ids", _I32),
+                  _addr(topk_w, "topk_w", _F32), _addr(perm, "perm", _I32),
+                  _addr(offsets, "offsets", _I32))
     if events is not None:
         for i, ev in enumerate(events):
             d.events[i] = None if ev is None else ev.cuda_event
@@ -189,8 +213,9 @@ def make_debug(logits=None, topk_ids=None, topk_w=None, perm=None, offsets=None,
 
 def moe_forward(plan, weights: moe_weights, hidden, valid, T: int, k: int, out, workspace,
                 ws_bytes: int, stream=None, dbg: moe_debug | None = None) -> None:
-    st = load().moe_forward(plan, ctypes.byref(weights), _addr(hidden), _addr(valid), T, k,
-                            _addr(out), _addr(workspace), ws_bytes, _stream(stream),
+    st = load().moe_forward(plan, ctypes.byref(weights), _addr(hidden, "hidden", _BF16),
+                            _addr(valid, "valid", _MASK), T, k, _addr(out, "out", _BF16),
+                            _addr(workspace, "workspace"), ws_bytes, _stream(stream),
                             None if dbg is None else ctypes.byref(dbg))
     _check(st, "moe_forward")
 
@@ -199,9 +224,10 @@ def moe_forward_scatter(plan, weights: moe_weights, hidden, valid, T: int, k: in
                         rows_per_rank: int, slot: int, workspace, ws_bytes: int, stream=None,
                         dbg: moe_debug | None = None) -> None:
     """dst: a sequence of device addresses (or tensors) of the owners' receive slabs."""
-    arr = (_vp * len(dst))(*[_addr(d) for d in dst])
-    st = load().moe_forward_scatter(plan, ctypes.byref(weights), _addr(hidden), _addr(valid), T, k,
-                                    arr, len(dst), rows_per_rank, slot, _addr(workspace),
+    arr = (_vp * len(dst))(*[_addr(d, "dst", _F32) for d in dst])
+    st = load().moe_forward_scatter(plan, ctypes.byref(weights), _addr(hidden, "hidden", _BF16),
+                                    _addr(valid, "valid", _MASK), T, k,
+                                    arr, len(dst), rows_per_rank, slot, _addr(workspace, "workspace"),
                                     ws_bytes, _stream(stream),
                                     None if dbg is None else ctypes.byref(dbg))
     _check(st, "moe_forward_scatter")
@@ -211,26 +237,32 @@ def moe_forward_scatter_experts(plan, weights: moe_weights, hidden, valid, T: in
                                 rows_per_rank: int, slot: int, expert_begin: int, expert_end: int,
                                 workspace, ws_bytes: int, stream=None,
                                 dbg: moe_debug | None = None) -> None:
-    arr = (_vp * len(dst))(*[_addr(d) for d in dst])
-    st = load().moe_forward_scatter_experts(plan, ctypes.byref(weights), _addr(hidden),
-                                            _addr(valid), T, k, arr, len(dst), rows_per_rank,
-                                            slot, expert_begin, expert_end, _addr(workspace),
+    arr = (_vp * len(dst))(*[_addr(d, "dst", _F32) for d in dst])
+    st = load().moe_forward_scatter_experts(plan, ctypes.byref(weights),
+                                            _addr(hidden, "hidden", _BF16),
+                                            _addr(valid, "valid", _MASK), T, k, arr, len(dst),
+                                            rows_per_rank, slot, expert_begin, expert_end,
+                                            _addr(workspace, "workspace"),
                                             ws_bytes, _stream(stream),
                                             None if dbg is None else ctypes.byref(dbg))
     _check(st, "moe_forward_scatter_experts")
 
 
 def moe_reduce_partials(slots, n_slots: int, rows: int, H: int, valid, out, stream=None) -> None:
-    st = load().moe_reduce_partials(_addr(slots), n_slots, rows, H, _addr(valid), _addr(out),
+    st = load().moe_reduce_partials(_addr(slots, "slots", _F32), n_slots, rows, H,
+                                    _addr(valid, "valid", _MASK), _addr(out, "out", _BF16),
                                     _stream(stream))
     _check(st, "moe_reduce_partials")
 
 
 def moe_route_from_logits(plan, logits, valid, T: int, k: int, topk_ids, topk_w, perm, offsets,
                           workspace, ws_bytes: int, stream=None) -> None:
-    st = load().moe_route_from_logits(plan, _addr(logits), _addr(valid), T, k, _addr(topk_ids),
-                                      _addr(topk_w), _addr(perm), _addr(offsets),
-                                      _addr(workspace), ws_bytes, _stream(stream))
+    st = load().moe_route_from_logits(plan, _addr(logits, "logits", _F32),
+                                      _addr(valid, "valid", _MASK), T, k,
+                                      _addr(topk_ids, "topk_ids", _I32),
+                                      _addr(topk_w, "topk_w", _F32), _addr(perm, "perm", _I32),
+                                      _addr(offsets, "offsets", _I32),
+                                      _addr(workspace, "workspace"), ws_bytes, _stream(stream))
     _check(st, "moe_route_from_logits")
 
 
@@ -238,16 +270,19 @@ def moe_route_from_logits_noalloc(plan, logits, valid, T: int, k: int, topk_ids,
                                   offsets, stream=None) -> None:
     """Routing from logits with the library's own static device scratch: for
     callers that cannot allocate device memory (no workspace argument)."""
-    st = load().moe_route_from_logits_noalloc(plan, _addr(logits), _addr(valid), T, k,
-                                              _addr(topk_ids), _addr(topk_w), _addr(perm),
-                                              _addr(offsets), _stream(stream))
+    st = load().moe_route_from_logits_noalloc(plan, _addr(logits, "logits", _F32),
+                                              _addr(valid, "valid", _MASK), T, k,
+                                              _addr(topk_ids, "topk_ids", _I32),
+                                              _addr(topk_w, "topk_w", _F32),
+                                              _addr(perm, "perm", _I32),
+                                              _addr(offsets, "offsets", _I32), _stream(stream))
     _check(st, "moe_route_from_logits_noalloc")
 
 
 def moe_check_device_status(plan, workspace, stream=None) -> int:
     """Returns the device status bits (0 = none); synchronises the stream."""
     bits = ctypes.c_uint32()
-    st = load().moe_check_device_status(plan, _addr(workspace), _stream(stream),
+    st = load().moe_check_device_status(plan, _addr(workspace, "workspace"), _stream(stream),
                                         ctypes.byref(bits))
     if st not in (MOE_OK, MOE_ERR_DEVICE):
         raise MoeError(st, "moe_check_device_status")
@@ -256,7 +291,7 @@ def moe_check_device_status(plan, workspace, stream=None) -> int:
 
 def moe_get_workspace_views(plan, workspace) -> moe_workspace_views:
     v = moe_workspace_views()
-    _check(load().moe_get_workspace_views(plan, _addr(workspace), ctypes.byref(v)),
+    _check(load().moe_get_workspace_views(plan, _addr(workspace, "workspace"), ctypes.byref(v)),
            "moe_get_workspace_views")
     return v
 
@@ -274,19 +309,74 @@ class Plan:
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8,
                                      device=device if device is not None else "cuda")
 
+    def weights(self, router_w, router_b=None, w_gate_up=None, w_down=None, s_gate_up=None,
+                s_down=None, ws_gate_up=None, ws_down=None, ss_gate_up=None,
+                ss_down=None) -> moe_weights:
+        """``make_weights`` with every tensor's shape checked against the plan: router
+        [E, H] (+ bias [E]), gate/up [E, 2I, H], down [E, H, I], FP8 block scales
+        [E, 2I/128, H/128] and [E, H/128, I/128], shared expert [2Is, H] / [H, Is] with
+        scales [2Is/128, H/128] / [H/128, Is/128] (a mis-shaped tensor would be read
+        past its end on the device).  Raw int addresses are taken as they are."""
+        c = self.cfg
+        E, H, I, Is = c.num_experts, c.hidden, c.inter, c.shared_inter
+        fp8 = c.wtype == MOE_W_FP8_E4M3_B128
+        want = {"router_w": (E, H), "w_gate_up": (E, 2 * I, H), "w_down": (E, H, I)}
+        optional = {"router_b": (E,)}
+        if fp8:
+            want.update(s_gate_up=(E, 2 * I // 128, H // 128), s_down=(E, H // 128, I // 128))
+        if c.num_shared:
+            want.update(ws_gate_up=(2 * Is, H), ws_down=(H, Is))
+            if fp8:
+                want.update(ss_gate_up=(2 * Is // 128, H // 128), ss_down=(H // 128, Is // 128))
+        given = dict(router_w=router_w, router_b=router_b, w_gate_up=w_gate_up, w_down=w_down,
+                     s_gate_up=s_gate_up, s_down=s_down, ws_gate_up=ws_gate_up,
+                     ws_down=ws_down, ss_gate_up=ss_gate_up, ss_down=ss_down)
+        for name, shape in {**want, **optional}.items():
+            t = given[name]
+            if t is None:
+                if name in want:
+                    raise ValueError(f"{name} is required by this plan")
+                continue
+            if not isinstance(t, int) and tuple(t.shape) != shape:
+                raise ValueError(f"{name}: shape {tuple(t.shape)}, the plan needs {shape}")
+        return make_weights(**given)
+
+    def _rows(self, hidden, valid, out=None) -> int:
+        """T of a call, after checking hidden [T, H], valid [T] and out [T, H]."""
+        H = self.cfg.hidden
+        if hidden.dim() != 2 or hidden.shape[1] != H:
+            raise ValueError(f"hidden: shape {tuple(hidden.shape)}, the plan needs [T, {H}]")
+        T = hidden.shape[0]
+        if valid is not None and tuple(valid.shape) != (T,):
+            raise ValueError(f"valid: shape {tuple(valid.shape)}, needs ({T},)")
+        if out is not None and tuple(out.shape) != (T, H):
+            raise ValueError(f"out: shape {tuple(out.shape)}, needs ({T}, {H})")
+        return T
+
+    def _slabs(self, dst, rows: int):
+        """Each receive slab tensor must hold len(dst) row blocks of ``rows`` rows."""
+        need = len(dst) * rows * self.cfg.hidden
+        for d in dst:
+            if not isinstance(d, int) and d.numel() < need:
+                raise ValueError(f"dst: a slab of {d.numel()} values, needs {need}")
+
     def forward(self, weights: moe_weights, hidden, valid, k: int, out, stream=None, dbg=None):
-        moe_forward(self.handle, weights, hidden, valid, hidden.shape[0], k, out, self.workspace,
-                    self.ws_bytes, stream, dbg)
+        moe_forward(self.handle, weights, hidden, valid, self._rows(hidden, valid, out), k, out,
+                    self.workspace, self.ws_bytes, stream, dbg)
 
     def forward_scatter(self, weights: moe_weights, hidden, valid, k: int, dst,
                         rows_per_rank: int, slot: int, stream=None, dbg=None):
-        moe_forward_scatter(self.handle, weights, hidden, valid, hidden.shape[0], k, dst,
+        T = self._rows(hidden, valid)
+        self._slabs(dst, rows_per_rank)
+        moe_forward_scatter(self.handle, weights, hidden, valid, T, k, dst,
                             rows_per_rank, slot, self.workspace, self.ws_bytes, stream, dbg)
 
     def forward_scatter_experts(self, weights: moe_weights, hidden, valid, k: int, dst,
                                 rows_per_rank: int, slot: int, expert_begin: int,
                                 expert_end: int, stream=None, dbg=None):
-        moe_forward_scatter_experts(self.handle, weights, hidden, valid, hidden.shape[0], k, dst,
+        T = self._rows(hidden, valid)
+        self._slabs(dst, rows_per_rank)
+        moe_forward_scatter_experts(self.handle, weights, hidden, valid, T, k, dst,
                                     rows_per_rank, slot, expert_begin, expert_end,
                                     self.workspace, self.ws_bytes, stream, dbg)
 
