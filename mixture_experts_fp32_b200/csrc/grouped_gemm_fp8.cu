@@ -15,13 +15,16 @@
 // buffers let the tensor core run one K block ahead of the promotion.
 //
 // One CTA per tile of 128 activation rows x 256 weight rows (M = 128, N = 256).
-// What bounds this loop is the hand-off of the two partial buffers: with a new
-// scale every 128 K, tensor memory (512 columns) holds two K blocks of partials,
-// and an MMA into a buffer must wait until the promotion has read it.  Tiles
-// of 256 rows on CTA pairs (cta_group::2, half the weight tile staged per CTA)
-// move less shared memory per K block but hit the same hand-off bound and pad
-// groups to 256 rows; measured on the 8192-token, 256-expert prefill they were
-// slower than this one-CTA form.
+// Two things bound this loop.  The larger is the operand feed: 48 KB of shared
+// memory per K block per CTA (a build of the same tile that accumulates all K
+// blocks in one buffer, i.e. without promotion, still runs at about 60 % of
+// the e4m3 rate on the 8192-token, 256-expert prefill).  The other is the
+// hand-off of the two partial buffers: with a new scale every 128 K, tensor
+// memory (512 columns) holds two K blocks of partials, and an MMA into a buffer
+// must wait until the promotion has read it (about a fifth of the time on that
+// workload).  Tiles of 256 rows on CTA pairs (cta_group::2, half the weight tile
+// staged per CTA) read less per K block but keep the hand-off and pad groups to
+// 256 rows; measured on the same prefill they were slower than this one-CTA form.
 //
 // Rows of activations take the MMA's M side and weight rows its N side: a TMEM
 // lane is one activation row, so the activation scale of a K block is one
