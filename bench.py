@@ -112,9 +112,16 @@ def algorithmic(w, valid_tokens: int, offsets, k: int):
     rows = routed_rows + S * valid_tokens
     gate_up_bytes = w_gate_up + rows * H * 2 + rows * max(I, Is) * 2
     gate_up_flops = 2 * routed_rows * 2 * I * H + 2 * valid_tokens * S * 2 * Is * H
+    # the design's intermediates, each written once and read once (not in the
+    # roofline): permuted rows x_perm, h, and the expert outputs y
+    if w.wtype == "bf16":
+        design_bytes = 2 * rows * (H * 2 + max(I, Is) * 2 + H * 4)
+    else:   # e4m3 rows with 1x128 fp32 scales, bf16 y
+        design_bytes = 2 * rows * (H + H // 128 * 4 + max(I, Is) + max(I, Is) // 128 * 4 + H * 2)
     return {"touched_experts": U, "routed_rows": routed_rows, "step_bytes": step_bytes,
             "step_flops": expert_flops + router_flops, "expert_flops": expert_flops,
-            "gate_up_bytes": gate_up_bytes, "gate_up_flops": gate_up_flops}
+            "gate_up_bytes": gate_up_bytes, "gate_up_flops": gate_up_flops,
+            "design_bytes": design_bytes}
 
 
 # ------------------------------------------------------------------- clocks
@@ -434,7 +441,10 @@ def run_native(args):
                               "frac_eager": step_roof_ms / ms,
                               "algorithmic_bytes": algo["step_bytes"],
                               "algorithmic_flops": algo["step_flops"],
-                              "touched_experts": algo["touched_experts"]},
+                              "touched_experts": algo["touched_experts"],
+                              "design_bytes": algo["design_bytes"],
+                              "design_ms_at_hbm": algo["design_bytes"]
+                              / (peaks["hbm_gbs"] * 1e9) * 1e3},
             "stage_ms": stage_ms,
             "step_ms_spread": {"rank": 0, "eager": step_spread(step_ms),
                                "graph": step_spread(gms) if graph_ms is not None else None,

@@ -58,3 +58,17 @@ def test_step_spread():
     s = bench.step_spread([float(v) for v in range(1, 12)])     # 1..11 ms
     assert s == {"p10": 2.0, "p50": 6.0, "p90": 10.0}
     assert bench.step_spread([]) == {"p10": None, "p50": None, "p90": None}
+
+
+def test_design_bytes():
+    # x_perm, h and y of every routed and shared row, written once and read once
+    w = synth.WORKLOADS["fp8_prefill"]
+    pairs = w.T * w.k
+    offsets = np.concatenate([[0], np.cumsum(np.full(w.E, pairs // w.E))])
+    a = bench.algorithmic(w, w.T, offsets, w.k)
+    R = pairs + w.T                                   # + the shared expert's rows
+    per_row = (7168 + 56 * 4) + (2048 + 16 * 4) + 7168 * 2
+    assert a["design_bytes"] == 2 * R * per_row       # about 3.5 GB
+    w = synth.WORKLOADS["step3_decode"]
+    a = bench.algorithmic(w, w.T, np.arange(0, 49 * 16, 16), w.k)
+    assert a["design_bytes"] == 2 * (768 + 256) * (7168 * 2 + 5120 * 2 + 7168 * 4)
