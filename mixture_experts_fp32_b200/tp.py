@@ -127,15 +127,43 @@ def split_rows(rows: int):
     return (0, a), (a, rows)
 
 
+class LibraryKernels:
+    """A rank's compute steps, run by the library on the GPU: the forward over the
+    gathered rows that stores each token's fp32 partial into the owners' slabs
+    (`moe_forward_scatter_experts`), and the owner's ordered sum and rounding
+    (`moe_reduce_partials`)."""
+
+    def __init__(self, shard: dict, *, E: int, H: int, inter: int, S: int, shared_inter: int,
+                 k_max: int, T: int, fp8: bool, device):
+        self.weights = make_shard_weights(shard)
+        self.plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
+                             inter=inter, num_shared=S, shared_inter=shared_inter,
+                             wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16,
+                             device=device)
+
+    def forward_scatter_experts(self, x_all, valid_all, k, dst, rows_per_rank, slot, e0, e1):
+        self.plan.forward_scatter_experts(self.weights, x_all, valid_all, k, dst, rows_per_rank,
+                                          slot, e0, e1)
+
+    def reduce_partials(self, slab, n_slots, rows, H, valid, out):
+        moe.moe_reduce_partials(slab, n_slots, rows, H, valid, out)
+
+
 class TPMoE:
     """One rank of the tensor-parallel layer (layout "tp") or of the expert-parallel one
     (layout "ep").  `full` holds the whole layer's weights on this rank's device (the
     shard is cut from it); `rows` is the number of rows each DP rank contributes per
-    micro-batch (padding rows included, marked invalid)."""
+    micro-batch (padding rows included, marked invalid).
+
+    ``kernels`` builds the compute steps from (shard, E, H, inter, S, shared_inter, k_max,
+    T, fp8, device); the default is the library (:class:`LibraryKernels`).  The
+    collectives, the row ownership and the slab layout are this class's own, so that a
+    stand-in for the two compute steps can run them on CPU ranks (the collective return
+    only: the fused one needs peer-mapped device memory)."""
 
     def __init__(self, full: dict, *, E: int, H: int, I: int, S: int, Is: int, k_max: int,
                  rows: int, fp8: bool = False, fused: bool = True, group=None,
-                 barrier_timeout_ms: int = 10000, layout: str = "tp"):
+                 barrier_timeout_ms: int = 10000, layout: str = "tp", kernels=LibraryKernels):
         import torch.distributed as dist
         self.group = group if group is not None else dist.group.WORLD
         self.n = dist.get_world_size(group)
@@ -152,12 +180,11 @@ class TPMoE:
             self.experts, inter = expert_range(E, self.n, self.rank), I
         else:
             raise ValueError(layout)
-        self.weights = make_shard_weights(self.shard)
         dev = full["w_gate_up"].device
         T = self.n * rows
-        self.plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
-                             inter=inter, num_shared=S, shared_inter=Is // self.n if S else 0,
-                             wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16, device=dev)
+        self.kernels = kernels(self.shard, E=E, H=H, inter=inter, S=S,
+                               shared_inter=Is // self.n if S else 0, k_max=k_max, T=T,
+                               fp8=fp8, device=dev)
         self.x_all = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.valid_all = torch.empty(T, dtype=torch.uint8, device=dev)
         self.step = 0
@@ -175,6 +202,10 @@ class TPMoE:
             self.partial = torch.empty(T, H, dtype=torch.float32, device=dev)
             self.recv = torch.empty(rows, H, dtype=torch.float32, device=dev)
 
+    @property
+    def plan(self):
+        return self.kernels.plan
+
     def _gather(self, x_local, valid_local):
         import torch.distributed as dist
         dist.all_gather_into_tensor(self.x_all, x_local, group=self.group)
@@ -184,19 +215,17 @@ class TPMoE:
         import torch.distributed as dist
         if self.fused:
             par = self.step & 1
-            self.plan.forward_scatter_experts(self.weights, self.x_all, self.valid_all, k,
-                                              self.dst[par], self.rows, self.rank,
-                                              *self.experts)
+            self.kernels.forward_scatter_experts(self.x_all, self.valid_all, k, self.dst[par],
+                                                 self.rows, self.rank, *self.experts)
             self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
-            moe.moe_reduce_partials(self.slab[par], self.n, self.rows, self.H, valid_local,
-                                    out_local)
+            self.kernels.reduce_partials(self.slab[par], self.n, self.rows, self.H, valid_local,
+                                         out_local)
         else:
-            self.plan.forward_scatter_experts(self.weights, self.x_all, self.valid_all, k,
-                                              [self.partial], self.n * self.rows, 0,
-                                              *self.experts)
+            self.kernels.forward_scatter_experts(self.x_all, self.valid_all, k, [self.partial],
+                                                 self.n * self.rows, 0, *self.experts)
             dist.reduce_scatter_tensor(self.recv, self.partial, op=dist.ReduceOp.SUM,
                                        group=self.group)
-            moe.moe_reduce_partials(self.recv, 1, self.rows, self.H, valid_local, out_local)
+            self.kernels.reduce_partials(self.recv, 1, self.rows, self.H, valid_local, out_local)
         self.step += 1
 
     def forward(self, x_local, valid_local, k: int, out_local):
