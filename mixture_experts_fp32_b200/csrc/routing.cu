@@ -323,7 +323,10 @@ __device__ __forceinline__ float elem8(const Vec8<__nv_bfloat16>& v, int i) {
   return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));   // bf16 -> fp32 is exact
 }
 
-template <typename YT, bool F32OUT>
+// MAXKS bounds k + S at compile time, so that the variant for up to four rows a token
+// (decode: top-3 with a shared expert) keeps only four row vectors in registers and
+// runs at twice the occupancy of the general one.
+template <typename YT, bool F32OUT, int MAXKS>
 __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, int H,
                                                       const int* __restrict__ inv,
                                                       const float* __restrict__ w,
@@ -360,22 +363,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, 
         const YT* yv = y + (size_t)v * 8;
 #define MOE_LD(J) \
   Vec8<YT> r##J;  \
-  if (J < ks && rows[J] >= 0) r##J = ld8(yv + (size_t)rows[J] * H);
+  if (J < MAXKS && J < ks && rows[J] >= 0) r##J = ld8(yv + (size_t)rows[J] * H);
         MOE_LD(0) MOE_LD(1) MOE_LD(2) MOE_LD(3) MOE_LD(4) MOE_LD(5) MOE_LD(6) MOE_LD(7) MOE_LD(8)
 #undef MOE_LD
 #define MOE_FMA(J)                                                                 \
-  if (J < k && rows[J] >= 0) {                                                     \
+  if (J < MAXKS && J < k && rows[J] >= 0) {                                        \
     _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] =                         \
         fmaf(wts[J], elem8(r##J, i), acc[i]);                                      \
   }
         MOE_FMA(0) MOE_FMA(1) MOE_FMA(2) MOE_FMA(3) MOE_FMA(4) MOE_FMA(5) MOE_FMA(6) MOE_FMA(7)
 #undef MOE_FMA
-        if (S && rows[k] >= 0) {                       // the shared expert's row, slot k
-          const Vec8<YT>& rs = k == 1 ? r1 : k == 2 ? r2 : k == 3 ? r3 : k == 4 ? r4
-                             : k == 5 ? r5 : k == 6 ? r6 : k == 7 ? r7 : r8;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += elem8(rs, i);
-        }
+        // the shared expert's row (slot k), added last
+#define MOE_SH(J)                                                                  \
+  if (J < MAXKS && S && J == k && rows[J] >= 0) {                                  \
+    _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] += elem8(r##J, i);        \
+  }
+        MOE_SH(1) MOE_SH(2) MOE_SH(3) MOE_SH(4) MOE_SH(5) MOE_SH(6) MOE_SH(7) MOE_SH(8)
+#undef MOE_SH
       }
       if (F32OUT) {
         dst32[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -530,15 +534,27 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* x, int H, const int* row_tok
   return cudaGetLastError();
 }
 
+// up to four rows a token (k + S <= 4) with the small-register variant
+template <typename YT, bool F32OUT>
+void launch_combine_rows(const YT* y, int H, const int* inv, const float* w,
+                         const uint8_t* valid, int T, int k, int S, const CombineOut& out,
+                         int grid, cudaStream_t st) {
+  if (k + S <= 4)
+    combine_kernel<YT, F32OUT, 4><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+  else
+    combine_kernel<YT, F32OUT, kMaxTopK + 1><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k,
+                                                                  S, out);
+}
+
 cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
                            const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                            cudaStream_t st) {
   int grid = T < 148 * 16 ? T : 148 * 16;
   if (grid < 1) grid = 1;
   if (out.bf16 != nullptr)
-    combine_kernel<float, false><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+    launch_combine_rows<float, false>(y, H, inv, w, valid, T, k, S, out, grid, st);
   else
-    combine_kernel<float, true><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+    launch_combine_rows<float, true>(y, H, inv, w, valid, T, k, S, out, grid, st);
   return cudaGetLastError();
 }
 
@@ -548,9 +564,9 @@ cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, 
   int grid = T < 148 * 16 ? T : 148 * 16;
   if (grid < 1) grid = 1;
   if (out.bf16 != nullptr)
-    combine_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+    launch_combine_rows<__nv_bfloat16, false>(y, H, inv, w, valid, T, k, S, out, grid, st);
   else
-    combine_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S, out);
+    launch_combine_rows<__nv_bfloat16, true>(y, H, inv, w, valid, T, k, S, out, grid, st);
   return cudaGetLastError();
 }
 
