@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1,   /* a null pointer, a size out of range, misalignment */
-    MOE_ERR_UNSUPPORTED = -2,   /* a shape or type this build does not implement */
+    MOE_ERR_UNSUPPORTED = -2,   /* a shape or type the library does not implement */
     MOE_ERR_WORKSPACE = -3,     /* workspace smaller than moe_plan_create reported */
     MOE_ERR_CUDA = -4,          /* a CUDA runtime call failed (launch, attribute, sync) */
     MOE_ERR_DEVICE = -5         /* moe_check_device_status found a device-side failure */

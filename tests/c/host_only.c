@@ -40,7 +40,7 @@ int main(void) {
   CHECK(moe_plan_create(&big, &plan2, &ws2) == MOE_OK && ws2 > ws);
   moe_plan_destroy(plan2);
 
-  /* shapes this build does not take are refused on the host */
+  /* shapes the library does not take are refused on the host */
   moe_config bad = cfg;
   bad.inter = 100;
   moe_plan_t p3 = NULL;
