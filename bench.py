@@ -489,7 +489,7 @@ def oracle_tokens_per_s(w, target_s: float):
     import synth
     inp = synth.make_inputs(w)
     valid_idx = np.nonzero(inp["valid"].numpy())[0]
-    cores = os.cpu_count() or 1
+    cores = oracle.max_threads()          # the threads the oracle's loops actually use
     n = min(len(valid_idx), max(1, cores))
     while True:
         tok = valid_idx[:n]

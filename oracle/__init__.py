@@ -64,8 +64,15 @@ def lib():
         L.oracle_moe_tokens_fp8.restype = None
         L.oracle_round_bf16.argtypes = [_P, ctypes.c_size_t, _P]
         L.oracle_round_bf16.restype = None
+        L.oracle_max_threads.argtypes = []
+        L.oracle_max_threads.restype = _I
         _lib = L
     return _lib
+
+
+def max_threads() -> int:
+    """Threads the oracle's token loops run on (OpenMP's current maximum)."""
+    return int(lib().oracle_max_threads())
 
 
 # ------------------------------------------------------------------ helpers

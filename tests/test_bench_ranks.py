@@ -76,3 +76,21 @@ def test_algorithmic_bytes_follow_touched_experts(name):
     b = bench.algorithmic(w, valid, np.maximum.accumulate(half), w.k)
     assert b["touched_experts"] < a["touched_experts"]
     assert b["step_bytes"] < a["step_bytes"]
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    import json
+    import oracle
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    args = bench.argparse.Namespace(workload="tiny", steps=2, warmup=0, cpu_seconds=0.2,
+                                    experts=0)
+    res = bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line == json.loads(json.dumps(res))
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"]
+    assert line["config"]["workload"] == "tiny" and line["n_gpus"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] == oracle.max_threads() >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
