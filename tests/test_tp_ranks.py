@@ -1,4 +1,4 @@
-"""The tensor- and expert-parallel layers' host side on two gloo ranks (CPU).
+"""The tensor- and expert-parallel layers' host side on two and four gloo ranks (CPU).
 
 TPMoE's own steps run for real: the all_gather of every rank's rows and masks, the
 collective return (reduce_scatter of the fp32 partials), the row ownership and each
@@ -27,8 +27,15 @@ WORKLOADS = {
                     bias="zipf"),
     "ep_fp8_no_shared": dict(T=2 * 16, H=256, E=4, k=2, I=128, S=0, Is=0, wtype="fp8",
                              router_sigma=0.2, w_sigma=0.05),
+    "tp_fp8": dict(T=2 * 16, H=256, E=8, k=2, I=256, S=1, Is=256, wtype="fp8",
+                   router_sigma=0.2, w_sigma=0.05),
+    "tp4_padded": dict(T=4 * 16, H=256, E=8, k=3, I=512, S=1, Is=512, router_sigma=0.2,
+                       mask="dp_padded", dp_rows=(16, 3, 0, 9)),
+    "ep4": dict(T=4 * 16, H=256, E=8, k=2, I=128, S=1, Is=512, router_sigma=0.2),
 }
-LAYOUT = {"tp_padded": "tp", "ep_zipf": "ep", "ep_fp8_no_shared": "ep"}
+LAYOUT = {"tp_padded": "tp", "ep_zipf": "ep", "ep_fp8_no_shared": "ep", "tp_fp8": "tp",
+          "tp4_padded": "tp", "ep4": "ep"}
+WORLD = {"tp4_padded": 4, "ep4": 4}
 
 
 class OracleKernels:
@@ -112,19 +119,20 @@ def _spawn(target, args_of, world=2):
 
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
-def test_two_ranks_return_the_layer(name):
+def test_ranks_return_the_layer(name):
     import oracle
     import synth
     from synth.workloads import Workload
-    procs, q = _spawn(_rank_main, lambda r: (name,))
-    got = dict(q.get(timeout=240) for _ in range(2))
+    world = WORLD.get(name, 2)
+    procs, q = _spawn(_rank_main, lambda r: (name,), world=world)
+    got = dict(q.get(timeout=240) for _ in range(world))
     for p in procs:
         p.join(60)
         assert p.exitcode == 0
     w = Workload(name, **WORKLOADS[name])
     inp = synth.make_inputs(w)
     ref = oracle.forward(inp)
-    out = np.concatenate([got[0], got[1]]).view(np.uint16)
+    out = np.concatenate([got[r] for r in range(world)]).view(np.uint16)
     ref_f = oracle.bf16_to_f64(ref["out"])
     out_f = oracle.bf16_to_f64(out)
     valid = inp["valid"].numpy().astype(bool)
