@@ -453,7 +453,8 @@ def run_native(args):
                     "ms_per_step": pipe_total / K,
                     "h2d_bytes_per_step": x_host.numel() * 2 + v_host.numel(),
                     "d2h_bytes_per_step": out_host.numel() * 2,
-                    "how": "HostPipeline: K steps back to back, each uploading its x and mask "
+                    "how": "the library's host-to-host pipeline (moe_pipeline_*, C ABI with "
+                           "host buffers): K steps back to back, each uploading its x and mask "
                            "from pinned host memory and downloading its output to pinned host "
                            "memory on copy streams beside the neighbouring steps' forwards "
                            "(3 slots" + (", graph replay" if args.graph else "") + "); L2 not "

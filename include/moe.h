@@ -270,6 +270,51 @@ typedef struct {
 } moe_workspace_views;
 moe_status moe_get_workspace_views(moe_plan_t plan, void *workspace, moe_workspace_views *views);
 
+/* Host-to-host forwards whose copies overlap the neighbouring batches' compute.
+ *
+ * A caller whose hidden states live in host memory pays, per batch, an upload of
+ * x and the mask and a download of out.  A pipeline runs them on two copy
+ * streams of its own beside a compute stream: the upload of batch i+1 and the
+ * download of batch i-1 proceed on the copy engines while batch i computes.
+ * Each of `depth` slots owns device buffers for one batch (x, mask, out, in
+ * caller-provided device memory); a slot is refilled only after its previous
+ * download has finished, and the forwards run one after another on the compute
+ * stream, so they share one workspace.  With three slots a step costs the
+ * longest of the forward, the upload and the download.
+ *
+ * moe_pipeline_slot_bytes: device bytes the slots of (plan, rows, depth) need.
+ * moe_pipeline_create: rows 1..max_tokens rows a batch, depth 1..8 slots, k as
+ *   for moe_forward; `weights` (the structure is copied; the tensors it points
+ *   to must stay valid and unchanged), `slots` (device, 256-byte aligned, at
+ *   least moe_pipeline_slot_bytes) and `workspace` are owned by the caller and
+ *   used by no one else while the pipeline lives.  With use_graph != 0 each
+ *   slot's forward is captured once as a CUDA graph and replayed.  Creation
+ *   synchronises the device (the weights the caller prepared are then ready) and
+ *   runs one forward per slot on all-padding rows.
+ * moe_pipeline_submit: enqueues one batch and returns: hidden bf16 [rows, H]
+ *   and valid uint8 [rows] (NULL = all valid) are read from host memory, out
+ *   bf16 [rows, H] is written to host memory; the caller keeps the inputs
+ *   unchanged and does not read out until the batch is done (for example after
+ *   moe_pipeline_synchronize).  Page-locked host memory lets the copies overlap;
+ *   pageable memory works but copies synchronously.
+ * moe_pipeline_synchronize: waits until every submitted batch's output is in
+ *   host memory.
+ * moe_pipeline_streams: the pipeline's upload, compute and download streams
+ *   (cudaStream_t as void*), for callers that order or time work against them.
+ * moe_pipeline_destroy: waits for the batches in flight, releases the streams,
+ *   events and graphs (not the caller's memory). */
+typedef struct moe_pipeline_s *moe_pipeline_t;
+moe_status moe_pipeline_slot_bytes(moe_plan_t plan, int rows, int depth, size_t *bytes);
+moe_status moe_pipeline_create(moe_plan_t plan, const moe_weights *weights, int k, int rows,
+                               int depth, int use_graph, void *slots, size_t slots_bytes,
+                               void *workspace, size_t ws_bytes, moe_pipeline_t *pipeline);
+moe_status moe_pipeline_submit(moe_pipeline_t pipeline, const void *hidden_host,
+                               const uint8_t *valid_host, void *out_host);
+moe_status moe_pipeline_synchronize(moe_pipeline_t pipeline);
+moe_status moe_pipeline_streams(moe_pipeline_t pipeline, void **upload, void **compute,
+                                void **download);
+void moe_pipeline_destroy(moe_pipeline_t pipeline);
+
 const char *moe_status_string(moe_status s);
 
 /* Text of the last CUDA runtime error behind an MOE_ERR_CUDA returned to this

@@ -34,7 +34,9 @@ STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm
 EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "moe_forward",
             "moe_forward_scatter", "moe_forward_scatter_experts", "moe_reduce_partials",
             "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
-            "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string")
+            "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string",
+            "moe_pipeline_slot_bytes", "moe_pipeline_create", "moe_pipeline_submit",
+            "moe_pipeline_synchronize", "moe_pipeline_streams", "moe_pipeline_destroy")
 MAX_TP_RANKS = 8
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -119,6 +121,21 @@ def load():
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_last_cuda_error_string.argtypes = []
     L.moe_last_cuda_error_string.restype = ctypes.c_char_p
+    L.moe_pipeline_slot_bytes.argtypes = [_vp, _c_int, _c_int, ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_pipeline_slot_bytes.restype = _c_int
+    L.moe_pipeline_create.argtypes = [_vp, ctypes.POINTER(moe_weights), _c_int, _c_int, _c_int,
+                                      _c_int, _vp, ctypes.c_size_t, _vp, ctypes.c_size_t,
+                                      ctypes.POINTER(_vp)]
+    L.moe_pipeline_create.restype = _c_int
+    L.moe_pipeline_submit.argtypes = [_vp, _vp, _vp, _vp]
+    L.moe_pipeline_submit.restype = _c_int
+    L.moe_pipeline_synchronize.argtypes = [_vp]
+    L.moe_pipeline_synchronize.restype = _c_int
+    L.moe_pipeline_streams.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                       ctypes.POINTER(_vp)]
+    L.moe_pipeline_streams.restype = _c_int
+    L.moe_pipeline_destroy.argtypes = [_vp]
+    L.moe_pipeline_destroy.restype = None
     _lib = L
     return L
 
@@ -287,6 +304,61 @@ def moe_check_device_status(plan, workspace, stream=None) -> int:
     if st not in (MOE_OK, MOE_ERR_DEVICE):
         raise MoeError(st, "moe_check_device_status")
     return bits.value
+
+
+def _host_addr(t, name: str, dtypes=None) -> int | None:
+    """Address of a host (CPU) tensor argument: contiguous, of one of ``dtypes``."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if t.is_cuda:
+        raise ValueError(f"{name}: a host tensor is required, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: a contiguous tensor is required")
+    if dtypes is not None and str(t.dtype).rsplit(".", 1)[-1] not in dtypes:
+        raise ValueError(f"{name}: element type {t.dtype} is not one of {', '.join(dtypes)}")
+    return t.data_ptr()
+
+
+def moe_pipeline_slot_bytes(plan, rows: int, depth: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().moe_pipeline_slot_bytes(plan, rows, depth, ctypes.byref(n)),
+           "moe_pipeline_slot_bytes")
+    return n.value
+
+
+def moe_pipeline_create(plan, weights: moe_weights, k: int, rows: int, depth: int,
+                        use_graph: bool, slots, slots_bytes: int, workspace, ws_bytes: int):
+    h = _vp()
+    _check(load().moe_pipeline_create(plan, ctypes.byref(weights), k, rows, depth,
+                                      int(bool(use_graph)), _addr(slots, "slots"), slots_bytes,
+                                      _addr(workspace, "workspace"), ws_bytes, ctypes.byref(h)),
+           "moe_pipeline_create")
+    return h.value
+
+
+def moe_pipeline_submit(pipeline, hidden_host, valid_host, out_host) -> None:
+    _check(load().moe_pipeline_submit(pipeline, _host_addr(hidden_host, "hidden_host", _BF16),
+                                      _host_addr(valid_host, "valid_host", _MASK),
+                                      _host_addr(out_host, "out_host", _BF16)),
+           "moe_pipeline_submit")
+
+
+def moe_pipeline_synchronize(pipeline) -> None:
+    _check(load().moe_pipeline_synchronize(pipeline), "moe_pipeline_synchronize")
+
+
+def moe_pipeline_streams(pipeline):
+    """(upload, compute, download) cudaStream_t handles as ints."""
+    u, c, d = _vp(), _vp(), _vp()
+    _check(load().moe_pipeline_streams(pipeline, ctypes.byref(u), ctypes.byref(c),
+                                       ctypes.byref(d)), "moe_pipeline_streams")
+    return u.value or 0, c.value or 0, d.value or 0
+
+
+def moe_pipeline_destroy(pipeline) -> None:
+    load().moe_pipeline_destroy(pipeline)
 
 
 def moe_get_workspace_views(plan, workspace) -> moe_workspace_views:

@@ -398,7 +398,7 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
 MOE_EXPORT moe_status moe_forward(moe_plan_t plan, const moe_weights* wts, const void* hidden,
                                   const uint8_t* valid, int T, int k, void* out, void* workspace,
                                   size_t ws_bytes, void* stream, moe_debug* dbg) {
-  if (out == nullptr || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (plan == nullptr || out == nullptr || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   moe::CombineOut co;
   memset(&co, 0, sizeof(co));
   co.bf16 = static_cast<__nv_bfloat16*>(out);
@@ -510,6 +510,205 @@ MOE_EXPORT moe_status moe_get_workspace_views(moe_plan_t plan, void* workspace,
   v->x_scale = fp8 ? at<float>(workspace, plan->off_sx) : nullptr;
   v->h_scale = fp8 ? at<float>(workspace, plan->off_sh) : nullptr;
   return MOE_OK;
+}
+
+// ------------------------------------------------------------------ pipeline
+// Host-to-host forwards: uploads and downloads on two copy streams, forwards on
+// a compute stream, one slot of device buffers per batch in flight.
+
+constexpr int kMaxPipelineDepth = 8;
+
+struct moe_pipeline_s {
+  moe_plan_t plan = nullptr;
+  moe_weights wts;
+  int k = 0, rows = 0, depth = 0;
+  bool graph = false;
+  uint8_t* slots = nullptr;
+  size_t stride = 0, off_valid = 0, off_out = 0;
+  void* workspace = nullptr;
+  size_t ws_bytes = 0;
+  cudaStream_t up = nullptr, compute = nullptr, down = nullptr;
+  cudaEvent_t loaded[kMaxPipelineDepth] = {};
+  cudaEvent_t computed[kMaxPipelineDepth] = {};
+  cudaEvent_t drained[kMaxPipelineDepth] = {};
+  cudaGraphExec_t exec[kMaxPipelineDepth] = {};
+  bool used[kMaxPipelineDepth] = {};
+  long long count = 0;
+};
+
+namespace {
+
+// per slot: x bf16 [rows, H], valid uint8 [rows], out bf16 [rows, H], each 256-byte aligned
+void pipeline_layout(const moe_plan_s* p, int rows, size_t* off_valid, size_t* off_out,
+                     size_t* stride) {
+  const size_t xb = align_up((size_t)rows * p->cfg.hidden * 2);
+  *off_valid = xb;
+  *off_out = xb + align_up((size_t)rows);
+  *stride = *off_out + xb;
+}
+
+void pipeline_release(moe_pipeline_s* q) {
+  for (int s = 0; s < kMaxPipelineDepth; ++s) {
+    if (q->exec[s] != nullptr) cudaGraphExecDestroy(q->exec[s]);
+    if (q->loaded[s] != nullptr) cudaEventDestroy(q->loaded[s]);
+    if (q->computed[s] != nullptr) cudaEventDestroy(q->computed[s]);
+    if (q->drained[s] != nullptr) cudaEventDestroy(q->drained[s]);
+  }
+  if (q->up != nullptr) cudaStreamDestroy(q->up);
+  if (q->compute != nullptr) cudaStreamDestroy(q->compute);
+  if (q->down != nullptr) cudaStreamDestroy(q->down);
+  delete q;
+}
+
+moe_status cuda_status(cudaError_t e) { return check_launch(e); }
+
+// slot s's forward on the compute stream (the moe_forward launch sequence)
+moe_status pipeline_forward(moe_pipeline_s* q, int s) {
+  uint8_t* base = q->slots + (size_t)s * q->stride;
+  moe::CombineOut co;
+  memset(&co, 0, sizeof(co));
+  co.bf16 = reinterpret_cast<__nv_bfloat16*>(base + q->off_out);
+  return forward_impl(q->plan, &q->wts, base, base + q->off_valid, q->rows, q->k, co, 0,
+                      q->plan->cfg.num_experts, q->workspace, q->ws_bytes, q->compute, nullptr);
+}
+
+}  // namespace
+
+MOE_EXPORT moe_status moe_pipeline_slot_bytes(moe_plan_t plan, int rows, int depth,
+                                              size_t* bytes) {
+  if (plan == nullptr || bytes == nullptr || rows < 1 || rows > plan->cfg.max_tokens ||
+      depth < 1 || depth > kMaxPipelineDepth)
+    return MOE_ERR_INVALID_ARG;
+  size_t ov = 0, oo = 0, stride = 0;
+  pipeline_layout(plan, rows, &ov, &oo, &stride);
+  *bytes = stride * (size_t)depth;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_pipeline_create(moe_plan_t plan, const moe_weights* wts, int k,
+                                          int rows, int depth, int use_graph, void* slots,
+                                          size_t slots_bytes, void* workspace, size_t ws_bytes,
+                                          moe_pipeline_t* pipeline) {
+  if (pipeline == nullptr) return MOE_ERR_INVALID_ARG;
+  *pipeline = nullptr;
+  if (wts == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  moe_status st = moe_pipeline_slot_bytes(plan, rows, depth, &need);
+  if (st != MOE_OK) return st;
+  if (k < 1 || k > plan->cfg.top_k_max) return MOE_ERR_INVALID_ARG;
+  if (slots == nullptr || (reinterpret_cast<uintptr_t>(slots) & (kAlign - 1)) != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (slots_bytes < need) return MOE_ERR_WORKSPACE;
+  st = check_common(plan, rows, k, workspace, ws_bytes);
+  if (st != MOE_OK) return st;
+
+  moe_pipeline_s* q = new (std::nothrow) moe_pipeline_s;
+  if (q == nullptr) return MOE_ERR_INVALID_ARG;
+  q->plan = plan;
+  q->wts = *wts;
+  q->k = k;
+  q->rows = rows;
+  q->depth = depth;
+  q->graph = use_graph != 0;
+  q->slots = static_cast<uint8_t*>(slots);
+  pipeline_layout(plan, rows, &q->off_valid, &q->off_out, &q->stride);
+  q->workspace = workspace;
+  q->ws_bytes = ws_bytes;
+
+  // the weights and buffers the caller prepared on any stream are ready after this
+  st = cuda_status(cudaDeviceSynchronize());
+  if (st == MOE_OK) st = cuda_status(cudaStreamCreateWithFlags(&q->up, cudaStreamNonBlocking));
+  if (st == MOE_OK)
+    st = cuda_status(cudaStreamCreateWithFlags(&q->compute, cudaStreamNonBlocking));
+  if (st == MOE_OK) st = cuda_status(cudaStreamCreateWithFlags(&q->down, cudaStreamNonBlocking));
+  for (int s = 0; s < depth && st == MOE_OK; ++s) {
+    st = cuda_status(cudaEventCreateWithFlags(&q->loaded[s], cudaEventDisableTiming));
+    if (st == MOE_OK)
+      st = cuda_status(cudaEventCreateWithFlags(&q->computed[s], cudaEventDisableTiming));
+    if (st == MOE_OK)
+      st = cuda_status(cudaEventCreateWithFlags(&q->drained[s], cudaEventDisableTiming));
+  }
+  // all-padding batches in every slot; the first forward of each runs outside any
+  // capture (kernel attributes are set on first use)
+  if (st == MOE_OK) st = cuda_status(cudaMemsetAsync(slots, 0, need, q->compute));
+  for (int s = 0; s < depth && st == MOE_OK; ++s) st = pipeline_forward(q, s);
+  if (st == MOE_OK) st = cuda_status(cudaStreamSynchronize(q->compute));
+  for (int s = 0; s < depth && st == MOE_OK && q->graph; ++s) {
+    st = cuda_status(cudaStreamBeginCapture(q->compute, cudaStreamCaptureModeThreadLocal));
+    if (st != MOE_OK) break;
+    const moe_status fs = pipeline_forward(q, s);
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(q->compute, &g);
+    if (fs != MOE_OK || ce != cudaSuccess || g == nullptr) {
+      if (g != nullptr) cudaGraphDestroy(g);
+      st = fs != MOE_OK ? fs : cuda_status(ce != cudaSuccess ? ce : cudaErrorUnknown);
+      break;
+    }
+    st = cuda_status(cudaGraphInstantiate(&q->exec[s], g, 0));
+    cudaGraphDestroy(g);
+  }
+  if (st == MOE_OK) st = cuda_status(cudaStreamSynchronize(q->compute));
+  if (st != MOE_OK) {
+    pipeline_release(q);
+    return st;
+  }
+  *pipeline = q;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_pipeline_submit(moe_pipeline_t q, const void* hidden_host,
+                                          const uint8_t* valid_host, void* out_host) {
+  if (q == nullptr || hidden_host == nullptr || out_host == nullptr) return MOE_ERR_INVALID_ARG;
+  const int s = (int)(q->count % q->depth);
+  uint8_t* base = q->slots + (size_t)s * q->stride;
+  const size_t xb = (size_t)q->rows * q->plan->cfg.hidden * 2;
+  // refill a slot only after its previous output has been downloaded (which
+  // itself followed that forward, the last reader of the slot's inputs)
+  moe_status st = MOE_OK;
+  if (q->used[s]) st = cuda_status(cudaStreamWaitEvent(q->up, q->drained[s], 0));
+  if (st == MOE_OK)
+    st = cuda_status(cudaMemcpyAsync(base, hidden_host, xb, cudaMemcpyHostToDevice, q->up));
+  if (st == MOE_OK)
+    st = cuda_status(valid_host != nullptr
+                         ? cudaMemcpyAsync(base + q->off_valid, valid_host, (size_t)q->rows,
+                                           cudaMemcpyHostToDevice, q->up)
+                         : cudaMemsetAsync(base + q->off_valid, 1, (size_t)q->rows, q->up));
+  if (st == MOE_OK) st = cuda_status(cudaEventRecord(q->loaded[s], q->up));
+  if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(q->compute, q->loaded[s], 0));
+  if (st == MOE_OK)
+    st = q->graph ? cuda_status(cudaGraphLaunch(q->exec[s], q->compute)) : pipeline_forward(q, s);
+  if (st == MOE_OK) st = cuda_status(cudaEventRecord(q->computed[s], q->compute));
+  if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(q->down, q->computed[s], 0));
+  if (st == MOE_OK)
+    st = cuda_status(
+        cudaMemcpyAsync(out_host, base + q->off_out, xb, cudaMemcpyDeviceToHost, q->down));
+  if (st == MOE_OK) st = cuda_status(cudaEventRecord(q->drained[s], q->down));
+  if (st != MOE_OK) return st;
+  q->used[s] = true;
+  ++q->count;
+  return MOE_OK;
+}
+
+MOE_EXPORT moe_status moe_pipeline_synchronize(moe_pipeline_t q) {
+  if (q == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaStreamSynchronize(q->down));
+}
+
+MOE_EXPORT moe_status moe_pipeline_streams(moe_pipeline_t q, void** upload, void** compute,
+                                           void** download) {
+  if (q == nullptr) return MOE_ERR_INVALID_ARG;
+  if (upload != nullptr) *upload = q->up;
+  if (compute != nullptr) *compute = q->compute;
+  if (download != nullptr) *download = q->down;
+  return MOE_OK;
+}
+
+MOE_EXPORT void moe_pipeline_destroy(moe_pipeline_t q) {
+  if (q == nullptr) return;
+  cudaStreamSynchronize(q->up);
+  cudaStreamSynchronize(q->compute);
+  cudaStreamSynchronize(q->down);
+  pipeline_release(q);
 }
 
 namespace moe {

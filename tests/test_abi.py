@@ -128,6 +128,52 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
         moe.moe_plan_destroy(plan)
 
 
+def test_pipeline_sizes_and_rejections_before_any_cuda_call(lib):
+    plan, ws = moe.moe_plan_create(cfg())
+    try:
+        H = 7168
+        a = lambda v: (v + 255) // 256 * 256                     # noqa: E731
+        for rows, depth in ((256, 3), (1, 1), (100, 8)):
+            stride = 2 * a(rows * H * 2) + a(rows)               # x, valid, out per slot
+            assert moe.moe_pipeline_slot_bytes(plan, rows, depth) == depth * stride
+        n = ctypes.c_size_t()
+        for rows, depth in ((0, 3), (257, 3), (16, 0), (16, 9)):
+            assert lib.moe_pipeline_slot_bytes(plan, rows, depth, ctypes.byref(n)) == \
+                moe.MOE_ERR_INVALID_ARG
+        w = moe.make_weights(0x1000, None, 0x2000, 0x3000, ws_gate_up=0x4000, ws_down=0x5000)
+        need = moe.moe_pipeline_slot_bytes(plan, 16, 3)
+        SL, WS = 0x200000, 0x100000
+        good = dict(w=ctypes.byref(w), k=3, rows=16, depth=3, slots=SL, nslots=need,
+                    workspace=WS, ws_bytes=ws)
+
+        def create(**kw):
+            g = dict(good)
+            g.update(kw)
+            h = ctypes.c_void_p(0x1234)
+            st = lib.moe_pipeline_create(plan, g["w"], g["k"], g["rows"], g["depth"], 1,
+                                         g["slots"], g["nslots"], g["workspace"], g["ws_bytes"],
+                                         ctypes.byref(h))
+            assert h.value is None                               # nothing created
+            return st
+
+        assert create(w=None) == moe.MOE_ERR_INVALID_ARG
+        assert create(k=0) == moe.MOE_ERR_INVALID_ARG
+        assert create(k=4) == moe.MOE_ERR_INVALID_ARG            # k > top_k_max
+        assert create(rows=257) == moe.MOE_ERR_INVALID_ARG
+        assert create(depth=9) == moe.MOE_ERR_INVALID_ARG
+        assert create(slots=None) == moe.MOE_ERR_INVALID_ARG
+        assert create(slots=SL + 16) == moe.MOE_ERR_INVALID_ARG  # not 256-byte aligned
+        assert create(nslots=need - 1) == moe.MOE_ERR_WORKSPACE
+        assert create(workspace=None) == moe.MOE_ERR_INVALID_ARG
+        assert create(ws_bytes=ws - 1) == moe.MOE_ERR_WORKSPACE
+        assert lib.moe_pipeline_submit(None, 0x10, None, 0x20) == moe.MOE_ERR_INVALID_ARG
+        assert lib.moe_pipeline_synchronize(None) == moe.MOE_ERR_INVALID_ARG
+        assert lib.moe_pipeline_streams(None, None, None, None) == moe.MOE_ERR_INVALID_ARG
+        lib.moe_pipeline_destroy(None)
+    finally:
+        moe.moe_plan_destroy(plan)
+
+
 def test_tensor_parallel_entry_points_reject_bad_arguments_before_launch(lib):
     plan, ws = moe.moe_plan_create(cfg())
     try:

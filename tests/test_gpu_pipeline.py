@@ -1,6 +1,6 @@
-"""Host-to-host forwards through HostPipeline (copies on their own streams, slots
-reused, optionally graph-replayed) give, batch for batch, the bits of the plain
-forward on the same inputs."""
+"""Host-to-host forwards through the library's pipeline (moe_pipeline_*, wrapped by
+HostPipeline: copies on their own streams, slots reused, optionally graph-replayed)
+give, batch for batch, the bits of the plain forward on the same inputs."""
 import pytest
 import torch
 
@@ -51,8 +51,9 @@ def test_pipeline_matches_plain_forward(graph, depth):
     pipe = HostPipeline(plan, wts, W.k, W.T, depth=depth, graph=graph)
     outs = [torch.full((W.T, W.H), float("nan"), dtype=torch.bfloat16).pin_memory()
             for _ in xs]
-    events = [pipe.submit(x, v, o) for x, v, o in zip(xs, vs, outs)]
-    events[-1].synchronize()
+    for x, v, o in zip(xs, vs, outs):
+        pipe.submit(x, v, o)
+    pipe.synchronize()
     pipe.close()
     assert plan.device_status() == 0
     for i, (o, r) in enumerate(zip(outs, refs)):
