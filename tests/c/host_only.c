@@ -72,6 +72,20 @@ int main(void) {
                                     NULL, NULL) == MOE_ERR_INVALID_ARG);   /* range past E */
   CHECK(moe_reduce_partials((const float *)0x8000, 0, 4, 7168, NULL, out, NULL) ==
         MOE_ERR_INVALID_ARG);
+  CHECK(moe_forward(NULL, &w, x, NULL, 16, 3, out, wsp, ws, NULL, NULL) == MOE_ERR_INVALID_ARG);
+
+  /* the host-buffer pipeline: slot sizes, and refusals before any CUDA call */
+  size_t slot_bytes = 0;
+  CHECK(moe_pipeline_slot_bytes(plan, 16, 3, &slot_bytes) == MOE_OK && slot_bytes > 0);
+  CHECK(moe_pipeline_slot_bytes(plan, 0, 3, &slot_bytes) == MOE_ERR_INVALID_ARG);
+  moe_pipeline_t pipe = (moe_pipeline_t)0x1;
+  CHECK(moe_pipeline_create(plan, &w, 3, 16, 3, 1, (void *)0x200000, slot_bytes - 1, wsp, ws,
+                            &pipe) == MOE_ERR_WORKSPACE && pipe == NULL);
+  CHECK(moe_pipeline_create(plan, &w, 4, 16, 3, 1, (void *)0x200000, slot_bytes, wsp, ws,
+                            &pipe) == MOE_ERR_INVALID_ARG && pipe == NULL);
+  CHECK(moe_pipeline_submit(NULL, x, NULL, out) == MOE_ERR_INVALID_ARG);
+  moe_pipeline_destroy(NULL);
+
   CHECK(moe_plan_set_wait_limit(NULL, 1) == MOE_ERR_INVALID_ARG);
   CHECK(moe_plan_set_wait_limit(plan, 5000000000ull) == MOE_OK);
 
