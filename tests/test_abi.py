@@ -221,3 +221,29 @@ def test_plain_c_caller(lib, tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stderr + out.stdout
     assert "passed" in out.stdout
+
+
+def test_ctypes_structures_match_the_header(tmp_path):
+    """The binding's structures have the C header's sizes and field offsets (a
+    mismatch would hand the library garbage pointers)."""
+    structs = {"moe_config": moe.moe_config, "moe_weights": moe.moe_weights,
+               "moe_debug": moe.moe_debug, "moe_workspace_views": moe.moe_workspace_views}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "moe.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe)])
+    got = {}
+    for line in subprocess.check_output([str(exe)], text=True).splitlines():
+        parts = line.split()
+        got[(parts[0], parts[1])] = int(parts[2])
+    for name, cls in structs.items():
+        assert got[(name, "size")] == ctypes.sizeof(cls), name
+        for field, _ in cls._fields_:
+            assert got[(name, field)] == getattr(cls, field).offset, (name, field)
