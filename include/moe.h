@@ -106,7 +106,10 @@ moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns);
  *  w_down     [E, H, I]
  *  s_gate_up  fp32 [E, 2I/128, H/128], s_down fp32 [E, H/128, I/128] (FP8 only)
  *  ws_gate_up [2Is, H], ws_down [H, Is], ss_* likewise: the shared expert
- *             (NULL when num_shared = 0). */
+ *             (NULL when num_shared = 0).
+ *  router_split  the bf16 split of router_w that moe_split_router_weights
+ *             wrote, or NULL: then every forward splits router_w again (into
+ *             the workspace) before the router GEMM. */
 typedef struct {
     const float *router_w;
     const float *router_b;
@@ -118,7 +121,27 @@ typedef struct {
     const void *ws_down;
     const float *ss_gate_up;
     const float *ss_down;
+    const void *router_split;
 } moe_weights;
+
+/* The router GEMM runs on the tensor cores (which multiply bf16, not fp32,
+ * operands) with the fp32 router weights split exactly into three bf16 parts,
+ * Wr = W1 + W2 + W3, each part the round-to-nearest bf16 of what the parts
+ * before it left; every product of a bf16 hidden value with a part is exact in
+ * fp32, so the logits are the fp32-accumulated products with the full fp32
+ * weights.  The split depends on the weights only: make it once when the
+ * weights are loaded (and again whenever router_w changes) and pass it as
+ * moe_weights.router_split, and no forward repeats it.
+ *
+ * moe_router_split_bytes: bytes of the split, 3 * E16 * H * 2 with E16 = E
+ *   rounded up to a multiple of 16 (0 for a NULL plan).
+ * moe_split_router_weights: writes the split of router_w (fp32 [E, H], device)
+ *   into split (device, 16-byte aligned, split_bytes at least the size above:
+ *   else MOE_ERR_WORKSPACE), bf16 [3][E16][H], rows past E zero; enqueued on
+ *   the stream. */
+size_t moe_router_split_bytes(moe_plan_t plan);
+moe_status moe_split_router_weights(moe_plan_t plan, const float *router_w, void *split,
+                                    size_t split_bytes, void *stream);
 
 /* Optional copies of intermediate results (device pointers, each may be NULL):
  *  logits    fp32 [T, E]   (0 in padding rows)
@@ -217,14 +240,18 @@ moe_status moe_route_from_logits(moe_plan_t plan, const float *logits, const uin
  * device pointers, or code that must not allocate because a CUDA graph is
  * being captured on its stream.
  *
- * Results are identical to moe_route_from_logits (same kernels, same order of
- * operations).  Its scratch (status word, group offsets, a logits copy, the
- * inverse permutation and the row -> token map) lives in one file-scope
+ * Results are identical to moe_route_from_logits, bit for bit: the same top-k
+ * kernel, and the single-block routing kernel that moe_route_from_logits also
+ * runs up to 1024 tokens (above 1024 the workspace path spreads the counting
+ * over three kernels; the result, a stable counting sort, is the same).  Its
+ * scratch (status word, group offsets, the inverse permutation and the
+ * row -> token map; the logits are not copied) lives in one file-scope
  * __device__ array of MOE_STATIC_SCRATCH_BYTES that every GPU which loads the
  * library holds until the process exits.  A call needs
- *   256 + a(4 (E + 2)) + a(4 T E) + 2 a(4 T (k + S))  bytes,  a(n) = n rounded up to 256,
- * and returns MOE_ERR_UNSUPPORTED, launching nothing, when that exceeds
- * MOE_STATIC_SCRATCH_BYTES.
+ *   256 + a(4 (E + 2)) + 2 a(4 T (k + S))  bytes,  a(n) = n rounded up to 256,
+ * (S = num_shared) and returns MOE_ERR_UNSUPPORTED, launching nothing, when
+ * that exceeds MOE_STATIC_SCRATCH_BYTES (E = 256, k = 8, S = 1: up to 58,232
+ * tokens).
  *  - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
@@ -233,8 +260,10 @@ moe_status moe_route_from_logits(moe_plan_t plan, const float *logits, const uin
  *    call's contents (each call clears what it needs cleared).  Calls whose
  *    work overlaps on the GPU — on two streams, or from two threads — race on
  *    it: order them on one stream.
- *  - Its device status word is inside the array too; this routing raises no
- *    device-side failure that moe_check_device_status would report.
+ *  - Its device status word is inside the array too, and nothing can set it:
+ *    the top-k kernel emits only ids in [0, E) for valid rows and -1 for
+ *    padding rows, which routing skips, so the out-of-range check of the
+ *    routing kernel never fires.
  * Arguments as in moe_route_from_logits; none of the output pointers may be NULL. */
 #define MOE_STATIC_SCRATCH_BYTES (4u << 20)
 moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float *logits,

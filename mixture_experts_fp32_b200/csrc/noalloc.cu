@@ -1,7 +1,10 @@
 // moe_route_from_logits_noalloc: routing from given logits for callers that
 // cannot allocate device memory (see include/moe.h).  The scratch that
 // moe_route_from_logits takes from the caller's workspace lives here, in one
-// file-scope device array; the kernels and their order are the same.
+// file-scope device array.  The results are identical to that call's: the same
+// top-k kernel, and the routing kernel that moe_route_from_logits runs up to
+// 1024 tokens (above that the workspace path splits the counting over parallel
+// kernels with the same deterministic result; here one block walks the chunks).
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -56,10 +59,9 @@ MOE_EXPORT moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float
     return MOE_ERR_INVALID_ARG;
   const size_t E = (size_t)c.num_experts, S = (size_t)c.num_shared;
   const size_t ks = (size_t)k + S;
-  // layout: status | group offsets | logits copy | inverse | row -> token
+  // layout: status | group offsets | inverse | row -> token (the logits are not copied)
   const size_t off_goff = 256;
-  const size_t off_logits = off_goff + round256(sizeof(int) * (E + 2));
-  const size_t off_inv = off_logits + round256(sizeof(float) * (size_t)T * E);
+  const size_t off_inv = off_goff + round256(sizeof(int) * (E + 2));
   const size_t off_rowtok = off_inv + round256(sizeof(int) * (size_t)T * ks);
   const size_t need = off_rowtok + round256(sizeof(int) * (size_t)T * ks);
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
@@ -71,9 +73,8 @@ MOE_EXPORT moe_status moe_route_from_logits_noalloc(moe_plan_t plan, const float
   unsigned int* status = reinterpret_cast<unsigned int*>(scratch);
   int* goff = reinterpret_cast<int*>(scratch + off_goff);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (moe::launch_topk(logits, 1, nullptr, valid, T, (int)E, k, c.renormalize,
-                       reinterpret_cast<float*>(scratch + off_logits), topk_ids, topk_w,
-                       st) != cudaSuccess)
+  if (moe::launch_topk(logits, 1, nullptr, valid, T, (int)E, k, c.renormalize, nullptr,
+                       topk_ids, topk_w, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (moe::launch_route(topk_ids, valid, T, (int)E, k, (int)S, 0, (int)E, goff, perm,
                         reinterpret_cast<int*>(scratch + off_inv),

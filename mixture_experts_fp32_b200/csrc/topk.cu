@@ -2,7 +2,8 @@
 // (MI308X vs H20), §背景: each token keeps 3 of 48 experts).
 //
 // topk_kernel: one warp per token.  It adds the router's split-K partial sums
-// in split order (plus the per-expert bias), keeps the logits, and runs k
+// in split order (plus the per-expert bias), keeps the logits (when logits_out
+// is not null), and runs k
 // rounds of a warp arg-max under the order (logit descending, expert
 // ascending); the weights are the softmax of the selected logits
 // (renormalised) or their full-softmax probabilities.
@@ -29,7 +30,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
   const int per_lane = (E + 31) / 32;   // <= 8
 
   if (valid != nullptr && !valid[t]) {
-    for (int e = lane; e < E; e += 32) logits_out[(size_t)t * E + e] = 0.f;
+    if (logits_out != nullptr)
+      for (int e = lane; e < E; e += 32) logits_out[(size_t)t * E + e] = 0.f;
     if (lane < k) {
       ids[(size_t)t * k + lane] = -1;
       w[(size_t)t * k + lane] = 0.f;
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
       for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * T + t) * E + e];
       if (bias != nullptr) s += bias[e];
       v[i] = s;
-      logits_out[(size_t)t * E + e] = s;
+      if (logits_out != nullptr) logits_out[(size_t)t * E + e] = s;
       avail |= 1u << i;
     }
   }
