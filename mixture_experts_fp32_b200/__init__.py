@@ -36,7 +36,8 @@ EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "m
             "moe_route_from_logits", "moe_route_from_logits_noalloc", "moe_check_device_status",
             "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string",
             "moe_pipeline_slot_bytes", "moe_pipeline_create", "moe_pipeline_submit",
-            "moe_pipeline_synchronize", "moe_pipeline_streams", "moe_pipeline_destroy")
+            "moe_pipeline_synchronize", "moe_pipeline_streams", "moe_pipeline_destroy",
+            "moe_router_split_bytes", "moe_split_router_weights")
 MAX_TP_RANKS = 8
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -54,7 +55,7 @@ class moe_config(ctypes.Structure):
 class moe_weights(ctypes.Structure):
     _fields_ = [("router_w", _vp), ("router_b", _vp), ("w_gate_up", _vp), ("w_down", _vp),
                 ("s_gate_up", _vp), ("s_down", _vp), ("ws_gate_up", _vp), ("ws_down", _vp),
-                ("ss_gate_up", _vp), ("ss_down", _vp)]
+                ("ss_gate_up", _vp), ("ss_down", _vp), ("router_split", _vp)]
 
 
 class moe_debug(ctypes.Structure):
@@ -134,6 +135,10 @@ def load():
     L.moe_pipeline_streams.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                        ctypes.POINTER(_vp)]
     L.moe_pipeline_streams.restype = _c_int
+    L.moe_router_split_bytes.argtypes = [_vp]
+    L.moe_router_split_bytes.restype = ctypes.c_size_t
+    L.moe_split_router_weights.argtypes = [_vp, _vp, _vp, ctypes.c_size_t, _vp]
+    L.moe_split_router_weights.restype = _c_int
     L.moe_pipeline_destroy.argtypes = [_vp]
     L.moe_pipeline_destroy.restype = None
     _lib = L
@@ -209,12 +214,23 @@ def moe_plan_set_wait_limit(plan, limit_ns: int) -> None:
 
 def make_weights(router_w, router_b=None, w_gate_up=None, w_down=None, s_gate_up=None,
                  s_down=None, ws_gate_up=None, ws_down=None, ss_gate_up=None,
-                 ss_down=None) -> moe_weights:
+                 ss_down=None, router_split=None) -> moe_weights:
     return moe_weights(_addr(router_w, "router_w", _F32), _addr(router_b, "router_b", _F32),
                        _addr(w_gate_up, "w_gate_up", _WEIGHT), _addr(w_down, "w_down", _WEIGHT),
                        _addr(s_gate_up, "s_gate_up", _F32), _addr(s_down, "s_down", _F32),
                        _addr(ws_gate_up, "ws_gate_up", _WEIGHT), _addr(ws_down, "ws_down", _WEIGHT),
-                       _addr(ss_gate_up, "ss_gate_up", _F32), _addr(ss_down, "ss_down", _F32))
+                       _addr(ss_gate_up, "ss_gate_up", _F32), _addr(ss_down, "ss_down", _F32),
+                       _addr(router_split, "router_split", _BF16))
+
+
+def moe_router_split_bytes(plan) -> int:
+    return int(load().moe_router_split_bytes(plan))
+
+
+def moe_split_router_weights(plan, router_w, split, split_bytes: int, stream=None) -> None:
+    _check(load().moe_split_router_weights(plan, _addr(router_w, "router_w", _F32),
+                                           _addr(split, "split", _BF16), split_bytes,
+                                           _stream(stream)), "moe_split_router_weights")
 
 
 def make_debug(logits=None, topk_ids=None, topk_w=None, perm=None, offsets=None,
@@ -383,12 +399,16 @@ class Plan:
 
     def weights(self, router_w, router_b=None, w_gate_up=None, w_down=None, s_gate_up=None,
                 s_down=None, ws_gate_up=None, ws_down=None, ss_gate_up=None,
-                ss_down=None) -> moe_weights:
+                ss_down=None, split_router=True, stream=None) -> moe_weights:
         """``make_weights`` with every tensor's shape checked against the plan: router
         [E, H] (+ bias [E]), gate/up [E, 2I, H], down [E, H, I], FP8 block scales
         [E, 2I/128, H/128] and [E, H/128, I/128], shared expert [2Is, H] / [H, Is] with
         scales [2Is/128, H/128] / [H/128, Is/128] (a mis-shaped tensor would be read
-        past its end on the device).  Raw int addresses are taken as they are."""
+        past its end on the device).  Raw int addresses are taken as they are.
+        With split_router, the router weights' bf16 split is made here once
+        (moe_split_router_weights, on ``stream``) into a tensor the returned
+        structure keeps alive, and forwards read it; make the weights again after
+        changing router_w."""
         c = self.cfg
         E, H, I, Is = c.num_experts, c.hidden, c.inter, c.shared_inter
         fp8 = c.wtype == MOE_W_FP8_E4M3_B128
@@ -411,7 +431,15 @@ class Plan:
                 continue
             if not isinstance(t, int) and tuple(t.shape) != shape:
                 raise ValueError(f"{name}: shape {tuple(t.shape)}, the plan needs {shape}")
-        return make_weights(**given)
+        if not split_router:
+            return make_weights(**given)
+        import torch
+        nbytes = moe_router_split_bytes(self.handle)
+        split = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=self.workspace.device)
+        moe_split_router_weights(self.handle, router_w, split, nbytes, stream)
+        w = make_weights(**given, router_split=split)
+        w._router_split = split          # the structure holds only its address
+        return w
 
     def _rows(self, hidden, valid, out=None) -> int:
         """T of a call, after checking hidden [T, H], valid [T] and out [T, H]."""

@@ -183,6 +183,25 @@ MOE_EXPORT moe_status moe_plan_set_wait_limit(moe_plan_t plan, uint64_t limit_ns
   return MOE_OK;
 }
 
+MOE_EXPORT size_t moe_router_split_bytes(moe_plan_t plan) {
+  if (plan == nullptr) return 0;
+  return (size_t)2 * 3 * (size_t)moe::router_padded_experts(plan->cfg.num_experts) *
+         (size_t)plan->cfg.hidden;
+}
+
+MOE_EXPORT moe_status moe_split_router_weights(moe_plan_t plan, const float* router_w,
+                                               void* split, size_t split_bytes, void* stream) {
+  if (plan == nullptr || router_w == nullptr || split == nullptr || !aligned16(router_w) ||
+      !aligned16(split))
+    return MOE_ERR_INVALID_ARG;
+  if (split_bytes < moe_router_split_bytes(plan)) return MOE_ERR_WORKSPACE;
+  moe_status s = ensure_device(plan);
+  if (s != MOE_OK) return s;
+  return check_launch(moe::launch_split_router_weights(
+      router_w, plan->cfg.num_experts, plan->cfg.hidden, static_cast<__nv_bfloat16*>(split),
+      plan->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 // The forward pass; `co` says where the combine writes (the bf16 output, or
 // fp32 partial rows of a tensor- / expert-parallel rank), and [eb, ee) which
 // routed experts this call computes (their weights are the ones given).
@@ -208,6 +227,7 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     return MOE_ERR_INVALID_ARG;
   if ((wts->router_b != nullptr && (reinterpret_cast<uintptr_t>(wts->router_b) & 3u)) != 0)
     return MOE_ERR_INVALID_ARG;
+  if (wts->router_split != nullptr && !aligned16(wts->router_split)) return MOE_ERR_INVALID_ARG;
   if (c.wtype == MOE_W_FP8_E4M3_B128 &&
       (wts->s_gate_up == nullptr || wts->s_down == nullptr ||
        (S && (wts->ss_gate_up == nullptr || wts->ss_down == nullptr))))
@@ -238,9 +258,17 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
   int splits = 1, kb_per_split = H / 64;
   moe::router_split_plan(T, E, H, plan->num_sms, &splits, &kb_per_split);
-  s = check_launch(moe::launch_router_logits_tc(
-      x, valid, T, H, wts->router_w, E, at<__nv_bfloat16>(workspace, plan->off_wsplit), partial,
-      splits, kb_per_split, plan->num_sms, status, st));
+  // the router weights' bf16 split: the caller's (written once by
+  // moe_split_router_weights), else made here in the workspace
+  const __nv_bfloat16* w3 = static_cast<const __nv_bfloat16*>(wts->router_split);
+  if (w3 == nullptr) {
+    auto* w3_ws = at<__nv_bfloat16>(workspace, plan->off_wsplit);
+    s = check_launch(moe::launch_split_router_weights(wts->router_w, E, H, w3_ws, plan->num_sms, st));
+    if (s != MOE_OK) return s;
+    w3 = w3_ws;
+  }
+  s = check_launch(moe::launch_router_logits_tc(x, valid, T, H, w3, E, partial, splits,
+                                                kb_per_split, status, st));
   if (s != MOE_OK) return s;
   record(dbg, 1, st);
   s = check_launch(moe::launch_topk(partial, splits, wts->router_b, valid, T, E, k, c.renormalize,

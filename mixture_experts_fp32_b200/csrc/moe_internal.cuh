@@ -90,13 +90,15 @@ cudaError_t launch_combine_bf16y(const __nv_bfloat16* y, int H, const int* inv, 
                                  cudaStream_t st);
 cudaError_t prepare_grouped_gemm_fp8_kernels();
 
-// Router logits on the tensor cores (router_tc.cu).  W3: scratch [3, E_pad, H]
-// bf16 for the exact three-part split of Wr; partial: [splits, T, E] fp32.
+// Router logits on the tensor cores (router_tc.cu).  W3: [3, E_pad, H] bf16,
+// the exact three-part split of Wr (launch_split_router_weights writes it);
+// partial: [splits, T, E] fp32.
 int router_padded_experts(int E);
+cudaError_t launch_split_router_weights(const float* Wr, int E, int H, __nv_bfloat16* W3,
+                                        int num_sms, cudaStream_t st);
 cudaError_t launch_router_logits_tc(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
-                                    const float* Wr, int E, __nv_bfloat16* W3, float* partial,
-                                    int splits, int kb_per_split, int num_sms,
-                                    unsigned int* status, cudaStream_t st);
+                                    const __nv_bfloat16* W3, int E, float* partial, int splits,
+                                    int kb_per_split, unsigned int* status, cudaStream_t st);
 cudaError_t prepare_router_kernel();
 cudaError_t launch_topk(const float* partial, int splits, const float* bias, const uint8_t* valid,
                         int T, int E, int k, int renorm, float* logits_out, int* ids, float* w,

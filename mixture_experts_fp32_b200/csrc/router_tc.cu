@@ -236,15 +236,17 @@ cudaError_t prepare_router_kernel() {
                               RSMEM);
 }
 
+cudaError_t launch_split_router_weights(const float* Wr, int E, int H, __nv_bfloat16* W3,
+                                        int num_sms, cudaStream_t st) {
+  split_router_weights_kernel<<<num_sms * 4, 256, 0, st>>>(Wr, E, router_padded_experts(E), H,
+                                                           W3);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits_tc(const __nv_bfloat16* x, const uint8_t* valid, int T, int H,
-                                    const float* Wr, int E, __nv_bfloat16* W3, float* partial,
-                                    int splits, int kb_per_split, int num_sms,
-                                    unsigned int* status, cudaStream_t st) {
+                                    const __nv_bfloat16* W3, int E, float* partial, int splits,
+                                    int kb_per_split, unsigned int* status, cudaStream_t st) {
   const int E_pad = router_padded_experts(E);
-  int grid = num_sms * 4;
-  split_router_weights_kernel<<<grid, 256, 0, st>>>(Wr, E, E_pad, H, W3);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   CUtensorMap tmX, tmW;
   if (!map_bf16_rows(&tmX, x, H, T) || !map_bf16_rows(&tmW, W3, H, (uint64_t)3 * E_pad))
     return cudaErrorInvalidValue;

@@ -110,10 +110,12 @@ def shard_experts(full: Dict[str, Optional[torch.Tensor]], n: int, r: int, *, E:
     return out
 
 
-def make_shard_weights(sh: Dict[str, Optional[torch.Tensor]]) -> moe.moe_weights:
+def make_shard_weights(sh: Dict[str, Optional[torch.Tensor]],
+                       router_split=None) -> moe.moe_weights:
     return moe.make_weights(sh["router_w"], sh.get("router_b"), sh["w_gate_up"], sh["w_down"],
                             sh.get("s_gate_up"), sh.get("s_down"), sh.get("ws_gate_up"),
-                            sh.get("ws_down"), sh.get("ss_gate_up"), sh.get("ss_down"))
+                            sh.get("ws_down"), sh.get("ss_gate_up"), sh.get("ss_down"),
+                            router_split)
 
 
 def owner_of(t: int, rows: int):
@@ -135,11 +137,16 @@ class LibraryKernels:
 
     def __init__(self, shard: dict, *, E: int, H: int, inter: int, S: int, shared_inter: int,
                  k_max: int, T: int, fp8: bool, device):
-        self.weights = make_shard_weights(shard)
         self.plan = moe.Plan(max_tokens=T, hidden=H, num_experts=E, top_k_max=k_max,
                              inter=inter, num_shared=S, shared_inter=shared_inter,
                              wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16,
                              device=device)
+        # the router weights' bf16 split, made once here rather than in every forward
+        nbytes = moe.moe_router_split_bytes(self.plan.handle)
+        self.router_split = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=device)
+        moe.moe_split_router_weights(self.plan.handle, shard["router_w"], self.router_split,
+                                     nbytes)
+        self.weights = make_shard_weights(shard, router_split=self.router_split)
 
     def forward_scatter_experts(self, x_all, valid_all, k, dst, rows_per_rank, slot, e0, e1):
         self.plan.forward_scatter_experts(self.weights, x_all, valid_all, k, dst, rows_per_rank,

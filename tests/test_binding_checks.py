@@ -59,8 +59,19 @@ def test_host_tensor_never_reaches_the_library():
         moe.make_weights(torch.zeros(8, 256))
 
 
+class _ShapeOnlyPlan(moe.Plan):
+    """A Plan without a library plan or GPU: only the host-side shape checks of
+    ``weights`` run (no router split is made)."""
+
+    def weights(self, *a, **kw):
+        return super().weights(*a, split_router=False, **kw)
+
+    def close(self):
+        pass
+
+
 def _plan(wtype=moe.MOE_W_BF16, S=1):
-    p = moe.Plan.__new__(moe.Plan)
+    p = _ShapeOnlyPlan.__new__(_ShapeOnlyPlan)
     p.cfg = moe.moe_config(64, 256, 8, 2, 128, S, 128 if S else 0, 1, wtype)
     return p
 

@@ -182,3 +182,44 @@ def test_intermediate_rows_against_fp64():
         yref = Wd @ h[r, :I].double()
         yerr = (y[r].double() - yref).abs().max().item()
         assert yerr <= 1e-2 * yref.abs().max().item() + 1e-6, (r, g, yerr)
+
+
+def test_router_split_made_once():
+    """moe_split_router_weights writes Wr = W1 + W2 + W3 exactly (each part a bf16,
+    the first the round-to-nearest bf16 of Wr, the later ones of the remainder,
+    rows past E zero), and a forward that reads it equals, bit for bit, one that
+    splits the router weights itself."""
+    w = W("split_once", T=100, H=384, E=20, k=3, I=128, S=1, Is=128, router_sigma=0.3)
+    inp = synth.make_inputs(w)
+    d = to_device(inp)
+    plan = plan_for(w)
+    nbytes = moe.moe_router_split_bytes(plan.handle)
+    E16 = (w.E + 15) // 16 * 16
+    assert nbytes == 3 * E16 * w.H * 2
+    split = torch.full((3, E16, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    moe.moe_split_router_weights(plan.handle, d["router_w"], split, nbytes)
+    with pytest.raises(moe.MoeError):
+        moe.moe_split_router_weights(plan.handle, d["router_w"], split, nbytes - 2)
+    torch.cuda.synchronize()
+    parts = split.cpu().double()
+    wr = inp["router_w"].double()
+    assert torch.equal(parts[:, : w.E].sum(0), wr)                    # exact, in fp64
+    assert torch.equal(split[0, : w.E].cpu(), inp["router_w"].to(torch.bfloat16))
+    assert torch.all(parts[:, w.E:] == 0)
+    # each later part is at most half an ulp of bf16 of what came before it
+    assert torch.all(parts[1].abs() <= parts[0].abs() * 2.0 ** -8)
+    assert torch.all(parts[2].abs() <= parts[1].abs() * 2.0 ** -8)
+
+    outs = []
+    for wts in (plan.weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
+                             ws_gate_up=d["ws_gate_up"], ws_down=d["ws_down"]),
+                plan.weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
+                             ws_gate_up=d["ws_gate_up"], ws_down=d["ws_down"],
+                             split_router=False)):
+        out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+        plan.forward(wts, d["x"], d["valid"], w.k, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert wts.router_split is None
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert plan.device_status() == 0
