@@ -4,10 +4,16 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl re
 
 One step = one moe_forward (router, top-k, permute, gather, gate/up GEMM,
 down GEMM, combine) over one batch of the workload, inputs resident in HBM.
-Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch
-(seeded by rank) against the same weights: data-parallel replicas, no
-collective on the data path ("scaling": "weak").  --impl reference times the
-CPU oracle on the host cores instead.
+Prints one JSON line (rank 0).  On one GPU the line is the Step3 decode step
+(the headline) and carries the other timed workloads (DeepSeek-style decode,
+the DP-padded gather batch, FP8 block-scale prefill) under "workloads", each
+measured the same way in the same run; --workload NAME times that one alone.
+Under torchrun (N > 1) the default is the tensor-parallel layer behind DP
+attention on the Step3 decode batch (all_gather of the ranks' rows, every
+rank 1/N of each expert's intermediate dimension, partial sums returned into
+the owners' slabs by the combine): strong scaling of the same batch.
+--replicas runs N independent data-parallel replicas instead.  --impl
+reference times the CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -26,11 +32,14 @@ if ROOT not in sys.path:
 
 METRIC = "MoE-layer tokens/s; % of HBM (decode) / tensor-core (prefill) roofline"
 DEFAULT_WORKLOAD = "step3_decode"
+# the default one-GPU run: the headline first, then the other timed workloads
+ALL_WORKLOADS = ("step3_decode", "deepseek_decode", "dp_padded", "fp8_prefill")
 L2_FLUSH_BYTES = 512 << 20
 
-# DRAM traffic / algorithmic bytes of one gate/up GEMM launch, from the ncu capture
-# summarised in profiles/grouped_gemm_step3_e8.md; it applies only to the kernel
-# source it was measured on (sha256 prefix), and "traffic" is null otherwise.
+# DRAM traffic / algorithmic bytes of one bf16 gate/up GEMM launch, from an ncu
+# capture of that kernel on the Step3 decode shape (8 experts, 1 GPU); it applies
+# only to the kernel source it was measured on (sha256 prefix), and "traffic" is
+# null otherwise.
 GEMM_TRAFFIC = {"sha256_prefix": "0ed45de09043589f", "gate_up_ratio": 0.998}
 
 
@@ -50,6 +59,73 @@ def measured_peaks():
             "source": "fallback"}
 
 
+def _time_loop(fn, burst_reps: int = 10, sustain_s: float = 3.0):
+    """Best single-call time over burst_reps calls, and the mean time per call of
+    calls issued back to back for about sustain_s seconds (CUDA events, ms)."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(burst_reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    n = max(8, int(sustain_s * 1e3 / max(best, 1e-3)))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    e1.synchronize()
+    return best, e0.elapsed_time(e1) / n
+
+
+def measure_fp8_peak(n: int = 8192, sustain_s: float = 3.0) -> dict:
+    """Dense e4m3 tensor-core rate on this GPU, measured with the library GEMM of
+    the framework (cuBLASLt through torch): an n^3 e4m3 x e4m3 -> bf16 product with
+    one fp32 scale per tensor, best of 10 (burst) and back to back for sustain_s
+    (sustained).  The same product with 1x128 activation and 128x128 weight block
+    scales (the layer's arithmetic) is timed beside it where torch offers it."""
+    import torch
+    import torch.nn.functional as F
+    g = torch.Generator(device="cuda").manual_seed(0)
+    a = (torch.randn(n, n, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn)
+    bt = (torch.randn(n, n, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn)
+    one = torch.ones((), device="cuda", dtype=torch.float32)
+    flops = 2.0 * n ** 3
+    res = {"shape": f"{n}x{n}x{n} e4m3 -> bf16", "how": "torch._scaled_mm (cuBLASLt)"}
+    best, sus = _time_loop(lambda: torch._scaled_mm(a, bt.t(), one, one,
+                                                    out_dtype=torch.bfloat16), sustain_s=sustain_s)
+    res["tensorwise_tflops"] = flops / (best * 1e-3) / 1e12
+    res["tensorwise_tflops_sustained"] = flops / (sus * 1e-3) / 1e12
+    try:
+        kb = n // 128
+        sa = torch.rand(kb, n, device="cuda", generator=g).add_(0.5).t()      # [n, n/128]
+        l4 = (kb + 3) // 4 * 4
+        sb = torch.rand(n // 128, l4, device="cuda", generator=g).add_(0.5).t()  # [l4, n/128]
+        ST, SW = F.ScalingType, F.SwizzleType
+
+        def blockwise():
+            return F.scaled_mm(a, bt.t(), [sa], [ST.BlockWise1x128], [sb],
+                               [ST.BlockWise128x128], [SW.NO_SWIZZLE], [SW.NO_SWIZZLE],
+                               None, torch.bfloat16)
+        best, sus = _time_loop(blockwise, sustain_s=min(sustain_s, 1.0))
+        res["blockwise_1x128_128x128_tflops"] = flops / (best * 1e-3) / 1e12
+        res["blockwise_1x128_128x128_tflops_sustained"] = flops / (sus * 1e-3) / 1e12
+    except Exception as ex:   # not offered by this torch / cuBLASLt build
+        res["blockwise_1x128_128x128_tflops"] = None
+        res["blockwise_error"] = f"{type(ex).__name__}: {str(ex)[:160]}"
+    del a, bt
+    torch.cuda.empty_cache()
+    return res
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -58,11 +134,12 @@ def dist_env():
 
 
 def launches_per_step(w) -> int:
-    """Kernels one forward launches: weight split + router + top-k, the permutation
-    (1 kernel up to 1024 rows, 3 above), the row gather (FP8: quantise-and-scatter),
-    the two GEMMs and the combine."""
+    """Kernels one forward launches: router + top-k, the permutation (1 kernel up to
+    1024 rows, 3 above), the row gather (FP8: quantise-and-scatter), the two GEMMs
+    and the combine.  The router weights' bf16 split is made once with the weights
+    (moe_split_router_weights), not per step."""
     route = 1 if w.T <= 1024 else 3
-    return 3 + route + 1 + 2 + 1
+    return 2 + route + 1 + 2 + 1
 
 
 def step_spread(ms) -> dict:
@@ -114,8 +191,8 @@ def algorithmic(w, valid_tokens: int, offsets, k: int):
     gate_up_flops = 2 * routed_rows * 2 * I * H + 2 * valid_tokens * S * 2 * Is * H
     # the design's intermediates, each written once and read once (not in the
     # roofline): permuted rows x_perm, h, and the expert outputs y
-    if w.wtype == "bf16":
-        design_bytes = 2 * rows * (H * 2 + max(I, Is) * 2 + H * 4)
+    if w.wtype == "bf16":      # bf16 x_perm, h in two bf16 parts, fp32 y
+        design_bytes = 2 * rows * (H * 2 + max(I, Is) * 4 + H * 4)
     else:   # e4m3 rows with 1x128 fp32 scales, bf16 y
         design_bytes = 2 * rows * (H + H // 128 * 4 + max(I, Is) + max(I, Is) // 128 * 4 + H * 2)
     return {"touched_experts": U, "routed_rows": routed_rows, "step_bytes": step_bytes,
@@ -178,32 +255,90 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 
+def setup_dist(ws_n: int, local: int):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if ws_n > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=datetime.timedelta(seconds=600))
+    else:
+        torch.cuda.set_device(0)
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def expert_load(offsets) -> dict:
+    """The realised routing: rows per routed expert (pairs), summarised."""
+    import numpy as np
+    c = np.diff(np.asarray(offsets, dtype=np.int64))
+    t = c[c > 0]
+    if t.size == 0:
+        return {"touched": 0}
+    return {"touched": int(t.size), "pairs": int(c.sum()), "max_rows": int(t.max()),
+            "min_rows_touched": int(t.min()), "mean_rows_touched": float(t.mean()),
+            "cv_touched": float(t.std() / t.mean()),
+            "top8_share": float(np.sort(c)[::-1][:8].sum() / max(1, c.sum()))}
+
+
 def run_native(args):
+    """One GPU (or --replicas: N data-parallel replicas, no collective on the data
+    path): every workload of the run measured in turn, the first one the headline."""
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_fp32_b200 as moe
+    from mixture_experts_fp32_b200 import build as lib_build
+
+    ws_n, rank, local = dist_env()
+    dev = setup_dist(ws_n, local)
+    if rank == 0:
+        lib_build.build()
+    if ws_n > 1:
+        dist.barrier()
+    moe.load()
+    peaks = measured_peaks()
+    names = [args.workload] if args.single else list(ALL_WORKLOADS)
+    fp8_peak = None
+    results = {}
+    for i, name in enumerate(names):
+        w = workload_of(args, name)
+        if w.wtype == "fp8" and fp8_peak is None and not args.no_fp8_peak:
+            fp8_peak = measure_fp8_peak()
+            fp8_peak = {kk: (reduce_over_ranks(v, "max", ws_n, dev)
+                             if isinstance(v, float) else v) for kk, v in fp8_peak.items()}
+        results[name] = measure_workload(args, w, dev, ws_n, rank, peaks, fp8_peak,
+                                         headline=(i == 0))
+        torch.cuda.empty_cache()
+    result = None
+    if rank == 0:
+        result = results[names[0]]["line"]
+        if len(names) > 1:
+            result["workloads"] = {n: results[n]["summary"] for n in names}
+        result["fp8_peak"] = fp8_peak
+        print(json.dumps(result), flush=True)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def measure_workload(args, w, dev, ws_n, rank, peaks, fp8_peak, headline: bool):
+    """Times one workload: eager steps with the library's stage events, the same
+    step replayed from a CUDA graph (the headline time), and for the headline the
+    end-to-end host-to-host figure; then the CPU-baseline leg (rank 0, one GPU),
+    which also reports the parity of sampled rows against the oracle."""
     import numpy as np
     import torch
     import torch.distributed as dist
 
     import mixture_experts_fp32_b200 as moe
     from mixture_experts_fp32_b200.pipeline import HostPipeline
-    from mixture_experts_fp32_b200 import build as lib_build
     import synth
 
-    ws_n, rank, local = dist_env()
-    if ws_n > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", init_method="env://",
-                                timeout=__import__("datetime").timedelta(seconds=600))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    if rank == 0:
-        lib_build.build()
-    if ws_n > 1:
-        dist.barrier()
-    moe.load()
-
-    w = workload_of(args)
     k = w.k
+    t_gen = time.perf_counter()
     # weights: drawn once (rank 0) and broadcast; activations: one batch per rank
     inp = synth.make_inputs(w, with_weights=(rank == 0))
     if ws_n > 1:
@@ -230,7 +365,11 @@ def run_native(args):
             if rank != 0:
                 d[kk] = torch.empty(sh[0], dtype=sh[1], device=dev)
             dist.broadcast(d[kk], src=0)
+    # the host copies the oracle leg needs (hidden states, mask, router; the
+    # weights it reads are these same tensors)
+    host = inp if (rank == 0 and ws_n == 1) else None
     del inp
+    t_gen = time.perf_counter() - t_gen
 
     plan = moe.Plan(max_tokens=w.T, hidden=w.H, num_experts=w.E, top_k_max=k, inter=w.I,
                     num_shared=w.S, shared_inter=w.Is if w.S else 0, device=dev,
@@ -253,8 +392,9 @@ def run_native(args):
         fwd(want_offsets=True)
     torch.cuda.synchronize()
     if plan.device_status() != 0:
-        raise RuntimeError("device status set during warm-up")
-    algo = algorithmic(w, valid_tokens, offsets.cpu().numpy(), k)
+        raise RuntimeError(f"{w.name}: device status set during warm-up")
+    off_host = offsets.cpu().numpy()
+    algo = algorithmic(w, valid_tokens, off_host, k)
 
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_NUM_STAGES + 1)]
@@ -283,18 +423,10 @@ def run_native(args):
         fwd(events=ev[i])
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
-    clock_info = clocks.stop()
-    if ws_n > 1:
-        dist.barrier()
-    step_ms = [ev[i][0].elapsed_time(ev[i][moe.MOE_NUM_STAGES]) for i in range(K)]
-    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(K))
-                for s, name in enumerate(moe.STAGE_NAMES)}
-    status = plan.device_status()
-    total_ms = sum(step_ms)
-    gemm_ms = stage_ms["gate_up_gemm"]
 
     # the same step replayed from a CUDA graph captured once (outside the timed region)
     graph_ms = None
+    gms = []
     if args.graph:
         out_g = torch.empty_like(out)
         cap = torch.cuda.Stream(device=dev)
@@ -308,7 +440,6 @@ def run_native(args):
         if ws_n > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        gms = []
         for _ in range(K):
             flush.zero_()
             e0 = torch.cuda.Event(enable_timing=True)
@@ -322,12 +453,144 @@ def run_native(args):
         if ws_n > 1:
             dist.barrier()
         if not torch.equal(out_g.view(torch.int16), out.view(torch.int16)):
-            raise RuntimeError("graph replay differs from the eager forward")
+            raise RuntimeError(f"{w.name}: graph replay differs from the eager forward")
         graph_ms = reduce_over_ranks(sum(gms), "max", ws_n, dev) / K
         del g
+    clock_info = clocks.stop()
+    if ws_n > 1:
+        dist.barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][moe.MOE_NUM_STAGES]) for i in range(K)]
+    stage_ms = {name: statistics.mean(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(K))
+                for s, name in enumerate(moe.STAGE_NAMES)}
+    status = plan.device_status()
+    total_ms = reduce_over_ranks(sum(step_ms), "max", ws_n, dev)
+    gemm_ms = stage_ms["gate_up_gemm"]
 
-    # end to end: pinned host input -> device, forward, result -> pinned host.
-    # Serial: each step's copies and forward one after another on one stream.
+    e2e = e2e_serial = e2e_ms = None
+    if headline:
+        e2e, e2e_serial, e2e_ms = end_to_end(args, w, d, plan, weights, out, k, flush, stream,
+                                             valid_tokens, ws_n, dev, HostPipeline)
+
+    # routing and outputs of this batch for the parity leg (one more forward)
+    gpu = None
+    if host is not None and not args.no_cpu_baseline:
+        dbg_t = {"logits": torch.empty(w.T, w.E, dtype=torch.float32, device=dev),
+                 "topk_ids": torch.empty(w.T, k, dtype=torch.int32, device=dev),
+                 "topk_w": torch.empty(w.T, k, dtype=torch.float32, device=dev)}
+        plan.forward(weights, d["x"], d["valid"], k, out, stream=stream,
+                     dbg=moe.make_debug(**dbg_t))
+        torch.cuda.synchronize()
+        gpu = {key: v.cpu() for key, v in dbg_t.items()}
+        gpu["out"] = out.cpu()
+    del d, weights, plan, flush, out
+    torch.cuda.empty_cache()
+
+    status = int(reduce_over_ranks(float(status), "max", ws_n, dev))
+    tokens = reduce_over_ranks(float(valid_tokens), "sum", ws_n, dev)
+    if rank != 0:
+        return None
+    fp8 = w.wtype == "fp8"
+    bound = "tensor" if fp8 else "hbm"
+    if fp8 and fp8_peak is not None:
+        mm_peak = fp8_peak["tensorwise_tflops"]
+        mm_sustained = fp8_peak["tensorwise_tflops_sustained"]
+        peak_source = "measured_fp8 (e4m3 GEMM of the same run, burst)"
+    elif fp8:
+        mm_peak = 2 * peaks["bf16_tflops"]
+        mm_sustained = 2 * (peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"])
+        peak_source = "2x measured bf16 (nominal dense ratio)"
+    else:
+        mm_peak = peaks["bf16_tflops"]
+        mm_sustained = peaks["bf16_tflops_sustained"]
+        peak_source = peaks["source"]
+    if bound == "hbm":
+        achieved = algo["gate_up_bytes"] / (gemm_ms * 1e-3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        frac_sus = None
+    else:
+        achieved = algo["gate_up_flops"] / (gemm_ms * 1e-3) / 1e12
+        peak, unit = mm_peak, "TFLOP/s"
+        frac_sus = achieved / mm_sustained if mm_sustained else None
+    traffic = None
+    if gemm_source_hash() == GEMM_TRAFFIC["sha256_prefix"] and not fp8:
+        traffic = GEMM_TRAFFIC["gate_up_ratio"] * algo["gate_up_bytes"]
+    ms = total_ms / K
+    # expert flops at the weights' dtype peak, router flops (fp32 logits on the
+    # bf16 tensor path) at the bf16 figure
+    step_roof_ms = max(algo["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                       algo["expert_flops"] / (mm_peak * 1e12)
+                       + (algo["step_flops"] - algo["expert_flops"]) / (peaks["bf16_tflops"] * 1e12)
+                       ) * 1e3
+    head_ms = graph_ms if graph_ms is not None else ms
+    cpu = None
+    if host is not None and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, host, gpu, args.cpu_seconds if headline else args.parity_seconds)
+    roofline = {"bound": bound, "kernel": ("grouped_gemm_fp8 gate/up + SwiGLU + h quantisation"
+                                           if fp8 else "grouped_gemm gate/up + SwiGLU"),
+                "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic, "algorithmic_bytes": algo["gate_up_bytes"],
+                "algorithmic_flops": algo["gate_up_flops"], "launch_ms": gemm_ms,
+                "peak_source": peak_source if bound == "tensor" else peaks["source"],
+                # the same kernel against the rate measured over seconds under the
+                # power cap (the timed steps run back to back)
+                "frac_of_sustained": frac_sus}
+    step_roof = {"ms": step_roof_ms, "frac": step_roof_ms / head_ms,
+                 "frac_eager": step_roof_ms / ms,
+                 "algorithmic_bytes": algo["step_bytes"], "algorithmic_flops": algo["step_flops"],
+                 "touched_experts": algo["touched_experts"],
+                 "design_bytes": algo["design_bytes"],
+                 "design_ms_at_hbm": algo["design_bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e3}
+    config = {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens, "H": w.H, "E": w.E,
+              "k": k, "I": w.I, "S": w.S, "Is": w.Is, "wtype": w.wtype,
+              "parallelism": f"dp{ws_n} replicas" if ws_n > 1 else "single GPU",
+              "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps, outside the "
+                    "step events; weights alone exceed L2"}
+    summary = {"ms_per_step": head_ms, "value": tokens / (head_ms * 1e-3), "unit": "tokens/s",
+               "eager_ms_per_step": ms, "timing": ("CUDA-graph replay" if graph_ms is not None
+                                                   else "eager"),
+               "config": config, "roofline": roofline, "step_roofline": step_roof,
+               "stage_ms": stage_ms, "clocks": clock_info,
+               "step_ms_spread": {"eager": step_spread(step_ms),
+                                  "graph": step_spread(gms) if gms else None},
+               "expert_load": expert_load(off_host),
+               "parity": None if cpu is None else cpu.get("parity"),
+               "gpu_launches": launches_per_step(w) * K, "device_status": status,
+               "input_generation_s": t_gen}
+    line = {
+        "metric": METRIC, "value": tokens / (head_ms * 1e-3) if K else 0.0,
+        "unit": "tokens/s", "n_gpus": ws_n, "steps": K, "warmup": max(args.warmup, 3),
+        "ms_per_step": head_ms, "higher_is_better": True, "scaling": "weak",
+        "timing": ("CUDA-graph replay of one captured forward per step"
+                   if graph_ms is not None else "eager forward per step"),
+        "eager": {"ms_per_step": ms, "value": tokens / (ms * 1e-3)},
+        "vs_baseline": None, "dtype": w.wtype, "data": "synthetic (Philox4x32-10, seed 0)",
+        "config": config, "roofline": roofline, "step_roofline": step_roof,
+        "stage_ms": stage_ms,
+        "step_ms_spread": {"rank": 0, "eager": step_spread(step_ms),
+                           "graph": step_spread(gms) if gms else None,
+                           "e2e_serial": step_spread(e2e_ms) if e2e_ms else None},
+        "e2e": e2e, "e2e_serial": e2e_serial,
+        "gpu_launches": launches_per_step(w) * K,
+        "graph_replay": None if graph_ms is None else {
+            "ms_per_step": graph_ms, "value": tokens / (graph_ms * 1e-3), "unit": "tokens/s"},
+        "clocks": clock_info, "device_status": status, "wall_s_timed_region": t_wall,
+        "expert_load": summary["expert_load"],
+        "parity": summary["parity"],
+        "cpu_baseline": cpu,
+    }
+    return {"line": line, "summary": summary}
+
+
+def end_to_end(args, w, d, plan, weights, out, k, flush, stream, valid_tokens, ws_n, dev,
+               HostPipeline):
+    """The step through the C ABI with host buffers: pinned host input -> device,
+    forward, result -> pinned host.  Serial: each step's copies and forward one
+    after another on one stream; pipelined (the e2e headline): the library's
+    host-to-host pipeline, copies on its own streams beside the neighbouring
+    steps' forwards."""
+    import torch
+    import torch.distributed as dist
+    K = args.steps
     x_host = d["x"].cpu().pin_memory()
     v_host = d["valid"].cpu().pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -353,9 +616,7 @@ def run_native(args):
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
 
-    # Pipelined (the headline e2e): HostPipeline runs every step's upload and
-    # download on copy streams beside the neighbouring steps' forwards; K steps
-    # back to back, timed from before the first upload to after the last download
+    # K steps back to back, timed from before the first upload to after the last download
     pipe = HostPipeline(plan, weights, k, w.T, depth=3, graph=args.graph)
     outs_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(3)]
     for i in range(3):
@@ -375,144 +636,169 @@ def run_native(args):
     pipe.close()
     if not torch.equal(outs_host[(K - 1) % 3].view(torch.int16), out.cpu().view(torch.int16)):
         raise RuntimeError("pipelined output differs from the eager forward")
-
-    total_ms = reduce_over_ranks(total_ms, "max", ws_n, dev)
     e2e_total = reduce_over_ranks(sum(e2e_ms), "max", ws_n, dev)
     pipe_total = reduce_over_ranks(pipe_ms, "max", ws_n, dev)
     tokens = reduce_over_ranks(float(valid_tokens), "sum", ws_n, dev)
-    status = int(reduce_over_ranks(float(status), "max", ws_n, dev))
-
-    peaks = measured_peaks()
-    prefill = w.wtype == "fp8"
-    bound = "tensor" if prefill else "hbm"
-    if bound == "hbm":
-        achieved = algo["gate_up_bytes"] / (gemm_ms * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        unit = "GB/s"
-    else:
-        achieved = algo["gate_up_flops"] / (gemm_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"] * (2 if w.wtype == "fp8" else 1)
-        unit = "TFLOP/s"
-    traffic = None
-    if gemm_source_hash() == GEMM_TRAFFIC["sha256_prefix"] and w.wtype == "bf16":
-        traffic = GEMM_TRAFFIC["gate_up_ratio"] * algo["gate_up_bytes"]
-    ms = total_ms / K
-    # expert flops at the weights' dtype peak (FP8: twice the measured bf16 figure,
-    # the nominal dense ratio), router flops (fp32 logits) at the bf16 figure
-    mm_peak = peaks["bf16_tflops"] * (2 if w.wtype == "fp8" else 1) * 1e12
-    step_roof_ms = max(algo["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
-                       algo["expert_flops"] / mm_peak
-                       + (algo["step_flops"] - algo["expert_flops"]) / (peaks["bf16_tflops"] * 1e12)
-                       ) * 1e3
-
-    result = None
-    if rank == 0:
-        cpu = cpu_baseline(w, args) if (ws_n == 1 and not args.no_cpu_baseline) else None
-        # headline: the step replayed from a CUDA graph (how a serving engine runs a
-        # decode step); the eager pass gives the per-stage breakdown and kernel times
-        head_ms = graph_ms if graph_ms is not None else ms
-        result = {
-            "metric": METRIC, "value": tokens / (head_ms * 1e-3) if K else 0.0,
-            "unit": "tokens/s", "n_gpus": ws_n, "steps": K, "warmup": max(args.warmup, 3),
-            "ms_per_step": head_ms, "higher_is_better": True, "scaling": "weak",
-            "timing": ("CUDA-graph replay of one captured forward per step"
-                       if graph_ms is not None else "eager forward per step"),
-            "eager": {"ms_per_step": ms, "value": tokens / (ms * 1e-3)},
-            "vs_baseline": None, "dtype": w.wtype, "data": "synthetic (Philox4x32-10, seed 0)",
-            "config": {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens, "H": w.H,
-                       "E": w.E, "k": k, "I": w.I, "S": w.S, "Is": w.Is,
-                       "parallelism": f"dp{ws_n} replicas" if ws_n > 1 else "single GPU",
-                       "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps, "
-                             "outside the step events; weights alone exceed L2"},
-            "roofline": {"bound": bound, "kernel": "grouped_gemm gate/up + SwiGLU",
-                         "achieved": achieved, "peak": peak, "unit": unit,
-                         "frac": achieved / peak, "traffic": traffic,
-                         "algorithmic_bytes": algo["gate_up_bytes"],
-                         "algorithmic_flops": algo["gate_up_flops"],
-                         "launch_ms": gemm_ms, "peak_source": peaks["source"],
-                         # the same kernel against the matmul rate measured over seconds
-                         # under the power cap (the timed steps run back to back)
-                         "frac_of_sustained": (achieved / (peaks["bf16_tflops_sustained"]
-                                                           * (2 if w.wtype == "fp8" else 1))
-                                               if bound == "tensor"
-                                               and peaks.get("bf16_tflops_sustained")
-                                               else None)},
-            "step_roofline": {"ms": step_roof_ms, "frac": step_roof_ms / head_ms,
-                              "frac_eager": step_roof_ms / ms,
-                              "algorithmic_bytes": algo["step_bytes"],
-                              "algorithmic_flops": algo["step_flops"],
-                              "touched_experts": algo["touched_experts"],
-                              "design_bytes": algo["design_bytes"],
-                              "design_ms_at_hbm": algo["design_bytes"]
-                              / (peaks["hbm_gbs"] * 1e9) * 1e3},
-            "stage_ms": stage_ms,
-            "step_ms_spread": {"rank": 0, "eager": step_spread(step_ms),
-                               "graph": step_spread(gms) if graph_ms is not None else None,
-                               "e2e_serial": step_spread(e2e_ms)},
-            "e2e": {"value": tokens / (pipe_total * 1e-3 / K), "unit": "tokens/s",
-                    "ms_per_step": pipe_total / K,
-                    "h2d_bytes_per_step": x_host.numel() * 2 + v_host.numel(),
-                    "d2h_bytes_per_step": out_host.numel() * 2,
-                    "how": "the library's host-to-host pipeline (moe_pipeline_*, C ABI with "
-                           "host buffers): K steps back to back, each uploading its x and mask "
-                           "from pinned host memory and downloading its output to pinned host "
-                           "memory on copy streams beside the neighbouring steps' forwards "
-                           "(3 slots" + (", graph replay" if args.graph else "") + "); L2 not "
-                           "flushed: every step streams its weights (far above L2) through it"},
-            "e2e_serial": {"value": tokens / (e2e_total * 1e-3 / K), "unit": "tokens/s",
-                           "ms_per_step": e2e_total / K,
-                           "how": "upload, eager forward and download one after another on "
-                                  "one stream, L2 flushed before each step"},
-            "gpu_launches": launches_per_step(w) * K,
-            "graph_replay": None if graph_ms is None else {
-                "ms_per_step": graph_ms, "value": tokens / (graph_ms * 1e-3),
-                "unit": "tokens/s"},
-            "clocks": clock_info,
-            "device_status": status,
-            "wall_s_timed_region": t_wall,
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(result), flush=True)
-    if ws_n > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    return result
+    e2e = {"value": tokens / (pipe_total * 1e-3 / K), "unit": "tokens/s",
+           "ms_per_step": pipe_total / K,
+           "h2d_bytes_per_step": x_host.numel() * 2 + v_host.numel(),
+           "d2h_bytes_per_step": out_host.numel() * 2,
+           "how": "the library's host-to-host pipeline (moe_pipeline_*, C ABI with "
+                  "host buffers): K steps back to back, each uploading its x and mask "
+                  "from pinned host memory and downloading its output to pinned host "
+                  "memory on copy streams beside the neighbouring steps' forwards "
+                  "(3 slots" + (", graph replay" if args.graph else "") + "); L2 not "
+                  "flushed: every step streams its weights (far above L2) through it"}
+    e2e_serial = {"value": tokens / (e2e_total * 1e-3 / K), "unit": "tokens/s",
+                  "ms_per_step": e2e_total / K,
+                  "how": "upload, eager forward and download one after another on "
+                         "one stream, L2 flushed before each step"}
+    return e2e, e2e_serial, e2e_ms
 
 
 # --------------------------------------------------------- the CPU oracle
 
-def oracle_tokens_per_s(w, target_s: float):
-    """Times the oracle (routing and expert FFN) on growing samples of the
-    workload's valid tokens until one sample takes about target_s seconds."""
+def oracle_sample(valid_idx, n: int):
+    """n valid tokens spread evenly over the batch (all of them when n >= len)."""
+    import numpy as np
+    if n >= len(valid_idx):
+        return valid_idx
+    return valid_idx[np.unique(np.linspace(0, len(valid_idx) - 1, n).round().astype(np.int64))]
+
+
+def oracle_pass(inp, tok, k: int):
+    """The oracle's layer (routing from its own logits) on the given tokens: the
+    timed unit of the CPU baseline.  Returns logits, ids, w and the float64
+    accumulators of those tokens."""
+    import oracle
+    x = inp["x"][tok]
+    v = inp["valid"][tok]
+    logits = oracle.router_logits(x, v, inp["router_w"], inp["router_b"])
+    ids, wt = oracle.topk(logits, v, k)
+    oracle.route(ids, v, inp["workload"].E)
+    sub = dict(inp)
+    sub["x"] = x
+    sub["valid"] = v
+    acc = oracle.moe_tokens(sub, ids, wt)
+    return logits, ids, wt, acc
+
+
+def oracle_timed(inp, k: int, target_s: float):
+    """Times the oracle on growing evenly spread samples of the valid tokens until
+    one sample takes about target_s / 4 or more; returns the last sample's rate."""
     import numpy as np
 
     import oracle
-    import synth
-    inp = synth.make_inputs(w)
     valid_idx = np.nonzero(inp["valid"].numpy())[0]
     cores = oracle.max_threads()          # the threads the oracle's loops actually use
     n = min(len(valid_idx), max(1, cores))
     while True:
-        tok = valid_idx[:n]
+        tok = oracle_sample(valid_idx, n)
         t0 = time.perf_counter()
-        sub = dict(inp)
-        sub["x"] = inp["x"][tok]
-        sub["valid"] = inp["valid"][tok]
-        logits = oracle.router_logits(sub["x"], sub["valid"], inp["router_w"], inp["router_b"])
-        ids, wt = oracle.topk(logits, sub["valid"], w.k)
-        oracle.route(ids, sub["valid"], w.E)
-        oracle.moe_tokens(sub, ids, wt)
+        res = oracle_pass(inp, tok, k)
         dt = time.perf_counter() - t0
         if dt >= target_s / 4 or n >= len(valid_idx):
-            return n / dt, n, dt, cores
+            return len(tok) / dt, tok, dt, cores, res
         n = min(len(valid_idx), int(n * max(2.0, target_s / max(dt, 1e-3))))
 
 
-def cpu_baseline(w, args):
-    rate, n, dt, cores = oracle_tokens_per_s(w, args.cpu_seconds)
-    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} valid tokens of {w.name} (all weights), {dt:.1f} s, "
-                      f"double-precision C with OpenMP over tokens"}
+def parity_of_sample(inp, tok, res, gpu, k: int, fp8: bool) -> dict:
+    """The GPU forward's rows of the sampled tokens against the oracle's:
+    logits within 1e-4 (|l| + rms) elementwise; routing identical, or different
+    only where the k-th and (k+1)-th logits lie within that tolerance; outputs
+    max |gpu - oracle| / rms (oracle rms over the sample) on the tokens routed
+    alike, against the layer's bound (2e-2 bf16, 6e-2 FP8)."""
+    import numpy as np
+
+    import oracle
+    logits, ids, _, acc = res
+    gl = gpu["logits"].numpy()[tok].astype(np.float64)
+    ol = logits.astype(np.float64)
+    rms_l = float(np.sqrt(np.mean(ol ** 2))) or 1.0
+    logit_err = float(np.max(np.abs(gl - ol) / (np.abs(ol) + rms_l)))
+    gids = gpu["topk_ids"].numpy()[tok]
+    same = np.all(gids == ids, axis=1)
+    mism = np.nonzero(~same)[0]
+    near = 0
+    for i in mism:
+        # a near-tie: at every slot where the two differ, the chosen experts' oracle
+        # logits lie within twice the 1e-4 logit tolerance of each other
+        js = np.nonzero(gids[i] != ids[i])[0]
+        gap = max(abs(ol[i][ids[i][j]] - ol[i][gids[i][j]]) for j in js)
+        if gap <= 2e-4 * (np.abs(ol[i]).max() + rms_l):
+            near += 1
+    ref = oracle.bf16_to_f64(oracle.round_bf16(acc))
+    out = oracle.bf16_to_f64(gpu["out"][tok])
+    rms = float(np.sqrt(np.mean(acc ** 2))) or 1.0
+    # against the exact (float64) layer output, as the parity tests measure it; and,
+    # for information, against the oracle's own bf16 rounding of it (one bf16 ulp
+    # of a large output element is itself 1-3 % of the rms)
+    err = float(np.max(np.abs(out[same] - acc[same]))) / rms if same.any() else None
+    err_r = float(np.max(np.abs(out[same] - ref[same]))) / rms if same.any() else None
+    bound = 6e-2 if fp8 else 2e-2
+    return {"tokens": int(len(tok)), "max_err_over_rms": err, "bound": bound,
+            "within_bound": bool(err is not None and err <= bound),
+            "max_err_vs_rounded_over_rms": err_r,
+            "logit_rel_err_max": logit_err, "routing_mismatch_tokens": int(len(mism)),
+            "routing_mismatch_near_tie": int(near),
+            "how": "GPU forward of the timed batch vs the oracle on its own logits (float64 "
+                   "accumulation before its final rounding), tokens spread evenly over the batch"}
+
+
+def cpu_baseline(w, inp, gpu, target_s: float):
+    """The oracle timed on the host cores on a bounded sample of the workload's
+    valid tokens (about target_s of CPU work); when the GPU forward's outputs are
+    given, the same oracle results give the sample's parity."""
+    rate, tok, dt, cores, res = oracle_timed(inp, w.k, target_s)
+    out = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{len(tok)} valid tokens of {w.name} spread over the batch (all "
+                     f"weights), {dt:.1f} s, double-precision C with OpenMP over tokens"}
+    if gpu is not None:
+        out["parity"] = parity_of_sample(inp, tok, res, gpu, w.k, w.wtype == "fp8")
+    return out
+
+
+def tp_reference_rows(d, w, rank: int, rows: int, dev):
+    """Rows [rank * rows, (rank + 1) * rows) of one GPU's plain forward of the whole
+    gathered batch, computed before the layer is sharded."""
+    import torch
+
+    import mixture_experts_fp32_b200 as moe
+    plan = moe.Plan(max_tokens=w.T, hidden=w.H, num_experts=w.E, top_k_max=w.k, inter=w.I,
+                    num_shared=w.S, shared_inter=w.Is if w.S else 0, device=dev,
+                    wtype=moe.MOE_W_BF16 if w.wtype == "bf16" else moe.MOE_W_FP8_E4M3_B128)
+    wts = plan.weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
+                       d.get("s_gate_up"), d.get("s_down"), d.get("ws_gate_up"),
+                       d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    plan.forward(wts, d["x"], d["valid"], w.k, out)
+    torch.cuda.synchronize()
+    if plan.device_status() != 0:
+        raise RuntimeError("device status set in the one-GPU reference forward")
+    mine = out[rank * rows:(rank + 1) * rows].clone()
+    del plan, wts, out
+    torch.cuda.empty_cache()
+    return mine
+
+
+def tp_check(out, ref, valid, n_ranks: int, fp8: bool) -> dict:
+    """This rank's rows of the sharded layer against the one-GPU forward: identical
+    bits on one rank; on several, max |diff| <= 2e-2 (bf16) / 6e-2 (FP8) x the rms of
+    the reference's valid rows, and padding rows +0.0 exactly."""
+    import torch
+    pad = valid == 0
+    pad_ok = bool(torch.all(out[pad].view(torch.int16) == 0).item()) if pad.any() else True
+    if n_ranks == 1:
+        same = bool(torch.equal(out.view(torch.int16), ref.view(torch.int16)))
+        return {"ok": same and pad_ok, "rule": "bit-identical to the one-GPU forward",
+                "identical": same, "padding_zero": pad_ok}
+    v = valid != 0
+    o, r = out[v].double(), ref[v].double()
+    rms = float(r.pow(2).mean().sqrt()) if r.numel() else 1.0
+    err = float((o - r).abs().max()) / (rms or 1.0) if r.numel() else 0.0
+    bound = 6e-2 if fp8 else 2e-2
+    return {"ok": err <= bound and pad_ok, "rule": f"max|diff| <= {bound} x rms",
+            "max_err_over_rms": err, "padding_zero": pad_ok}
 
 
 def run_tp(args):
@@ -548,19 +834,27 @@ def run_tp(args):
             lib_build.build()
         dist.barrier()
         moe.load()
-        w = workload_of(args)
+        w = workload_of(args, args.workload)
         if w.T % ws_n:
             raise SystemExit(f"{w.T} rows do not split over {ws_n} ranks")
         rows = w.T // ws_n
         inp = synth.make_inputs(w)        # the same seeded layer and gathered batch on every rank
         d = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
         del inp
-        layer = tp.TPMoE(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is if w.S else 0, k_max=w.k,
-                         rows=rows, fp8=w.wtype == "fp8", fused=args.tp_return == "fused",
-                         layout=args.tp_layout)
+        valid_tokens = int(d["valid"].sum().item())
+        # the reference for this rank's rows: one GPU's plain forward of the gathered batch
+        ref_rows = tp_reference_rows(d, w, rank, rows, dev)
+        pairs = args.tp_return == "pairs"
+        kw = dict(E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is if w.S else 0, k_max=w.k,
+                  fp8=w.wtype == "fp8", fused=args.tp_return != "nccl",
+                  layout="ep" if pairs else args.tp_layout, pairs=pairs,
+                  send_ctas=args.send_ctas)
+        if args.tp_microbatches == 2 and rows >= 2:
+            layer = tp.TPMoETwoBatch(d, rows=rows, **kw)
+        else:
+            layer = tp.TPMoE(d, rows=rows, **kw)
         x_loc = d["x"][rank * rows:(rank + 1) * rows].contiguous()
         v_loc = d["valid"][rank * rows:(rank + 1) * rows].contiguous()
-        valid_tokens = int(d["valid"].sum().item())
         for key in ("w_gate_up", "w_down", "ws_gate_up", "ws_down", "s_gate_up", "s_down",
                     "ss_gate_up", "ss_down"):
             d[key] = None                                  # the shard keeps its own copy
@@ -571,8 +865,18 @@ def run_tp(args):
             flush.zero_()
             layer.forward(x_loc, v_loc, w.k, out)
         torch.cuda.synchronize()
-        if layer.plan.device_status() != 0:
+        plans = [h.plan for h in layer.halves] if hasattr(layer, "halves") else [layer.plan]
+        if any(p.device_status() != 0 for p in plans):
             raise RuntimeError("device status set during warm-up")
+        # every rank's own rows against the one-GPU forward, agreed on by all ranks
+        # before anything is timed (bit for bit on one rank; on several the partial
+        # sums are added in another order, so within the layer's tolerance)
+        check = tp_check(out, ref_rows, v_loc, ws_n, w.wtype == "fp8")
+        flag = torch.tensor([0.0 if check["ok"] else 1.0], device=dev)
+        if ws_n > 1:
+            dist.all_reduce(flag, op=dist.ReduceOp.MAX)
+        if flag.item() != 0.0:
+            raise RuntimeError(f"tensor-parallel rows differ from the one-GPU forward: {check}")
         K = args.steps
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
@@ -590,7 +894,7 @@ def run_tp(args):
         clk = clocks.stop()
         ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
         ms = reduce_over_ranks(ms, "max", ws_n, dev)
-        if layer.plan.device_status() != 0:
+        if any(p.device_status() != 0 for p in plans):
             raise RuntimeError("device status set during the timed steps")
         if rank == 0:
             print(json.dumps({
@@ -601,10 +905,13 @@ def run_tp(args):
                 "timing": "eager TP forward per step (all_gather, layer, partial return, reduce)",
                 "config": {"workload": w.name, "T": w.T, "valid_tokens": valid_tokens,
                            "rows_per_rank": rows, "H": w.H, "E": w.E, "k": w.k, "I": w.I,
-                           "S": w.S, "parallelism": f"{args.tp_layout}{ws_n}",
+                           "S": w.S, "parallelism": ("ep" if pairs else args.tp_layout)
+                                                       + str(ws_n),
                            "partial_return": args.tp_return,
+                           "send_ctas": args.send_ctas if pairs else None,
+                           "micro_batches": 2 if hasattr(layer, "halves") else 1,
                            "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps"},
-                "clocks": clk}))
+                "check": check, "gpu_launches": None, "clocks": clk}))
     finally:
         del layer
         torch.cuda.synchronize()
@@ -613,36 +920,56 @@ def run_tp(args):
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle (there is no installable reference
+    implementation; the pages hold no code) on the host cores, rank 0 only.  Each
+    step times the oracle on one bounded, evenly spread sample of the workload's
+    valid tokens, sized so that the whole --steps/--warmup run ends within a few
+    minutes; warm-up steps run a small sample."""
+    import numpy as np
+
+    import synth
     ws_n, rank, _ = dist_env()
     if rank != 0:
         return None
-    w = workload_of(args)
-    rates = []
+    w = workload_of(args, args.workload)
+    inp = synth.make_inputs(w)
+    valid_idx = np.nonzero(inp["valid"].numpy())[0]
+    per_step = max(1.0, min(args.cpu_seconds, args.reference_seconds /
+                            max(1, args.steps + args.warmup // 4 + 1)))
+    rate, tok, dt, cores, _ = oracle_timed(inp, w.k, per_step)   # calibrates the sample
+    small = oracle_sample(valid_idx, max(1, len(tok) // 8))
     for _ in range(max(args.warmup, 0)):
-        oracle_tokens_per_s(w, min(args.cpu_seconds, 5.0))
-    n = dt = cores = 0
+        oracle_pass(inp, small, w.k)
+    rates, times = [], []
     for _ in range(args.steps):
-        r, n, dt, cores = oracle_tokens_per_s(w, args.cpu_seconds)
-        rates.append(r)
+        t0 = time.perf_counter()
+        oracle_pass(inp, tok, w.k)
+        dt = time.perf_counter() - t0
+        times.append(dt)
+        rates.append(len(tok) / dt)
     value = statistics.median(rates) if rates else 0.0
     res = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * n / value if value else 0,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * statistics.median(times) if times else 0.0,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (Philox4x32-10, seed 0)", "impl": "reference",
-           "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k, "I": w.I,
-                      "S": w.S, "Is": w.Is},
+           "config": {"workload": w.name, "T": w.T, "valid_tokens": int(len(valid_idx)),
+                      "H": w.H, "E": w.E, "k": w.k, "I": w.I, "S": w.S, "Is": w.Is,
+                      "wtype": w.wtype, "parallelism": "single GPU"},
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                             "kind": "oracle",
-                            "sample": f"{n} valid tokens per step of {w.name}, {dt:.1f} s"},
+                            "sample": f"{len(tok)} valid tokens of {w.name} per step, spread "
+                                      f"over the batch (all weights); warm-up steps "
+                                      f"{len(small)} tokens"},
            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
     return res
 
 
-def workload_of(args):
+def workload_of(args, name: str):
     import synth
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[name]
     if args.experts:
         # a smaller copy of the workload (fewer experts) for profiler captures
         w = w.with_(name=f"{w.name}_e{args.experts}", E=args.experts, k=min(w.k, args.experts))
@@ -654,26 +981,46 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None,
+                    help="time this workload alone (default on one GPU: all timed workloads, "
+                         "the Step3 decode step as the headline)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU work of the headline's CPU-baseline sample")
+    ap.add_argument("--parity-seconds", type=float, default=4.0,
+                    help="CPU work of the oracle sample of each other workload")
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="budget of the reference arm's timed steps together")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8-peak", action="store_true")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager forwards only (default: the headline is CUDA-graph replay)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="under torchrun: N independent data-parallel replicas instead of "
+                         "the tensor-parallel layer")
     ap.add_argument("--tp", action="store_true",
-                    help="tensor-parallel layout over the N ranks (default workload: dp_padded)")
-    ap.add_argument("--tp-return", default="fused", choices=["fused", "nccl"])
+                    help="tensor-parallel layout over the N ranks (the default under torchrun; "
+                         "with --tp alone the workload defaults to dp_padded)")
+    ap.add_argument("--tp-return", default="fused", choices=["fused", "nccl", "pairs"],
+                    help="fused: the combine stores each token's partial into its owner's "
+                         "slab; nccl: reduce_scatter; pairs: expert-parallel per-pair return "
+                         "from sender CTAs signalled by the down GEMM")
+    ap.add_argument("--send-ctas", type=int, default=16,
+                    help="with --tp-return pairs: CTAs of the down GEMM launch that send")
     ap.add_argument("--tp-layout", default="tp", choices=["tp", "ep"],
                     help="with --tp: split every expert's intermediate dimension (tp) or "
                          "the experts (ep) over the ranks")
+    ap.add_argument("--tp-microbatches", type=int, default=2, choices=[1, 2])
     ap.add_argument("--experts", type=int, default=0,
                     help="override the number of routed experts (profiling on a smaller case)")
     args = ap.parse_args(argv)
-    if args.tp and args.workload == DEFAULT_WORKLOAD and "--workload" not in (argv or sys.argv):
-        args.workload = "dp_padded"
+    ws_n = dist_env()[0]
+    args.single = args.workload is not None or args.experts > 0
+    if args.workload is None:
+        args.workload = "dp_padded" if args.tp else DEFAULT_WORKLOAD
     if args.impl == "reference":
         run_reference(args)
-    elif args.tp:
+    elif args.tp or (ws_n > 1 and not args.replicas):
         run_tp(args)
     else:
         run_native(args)

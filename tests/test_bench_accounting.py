@@ -47,11 +47,11 @@ def test_untouched_experts_cost_no_weight_bytes():
 
 
 def test_launch_count_per_step():
-    # weight split, router, top-k; the permutation (1 kernel up to 1024 rows, 3 above);
-    # the gather or FP8 quantisation; two GEMMs; the combine. The decode figure is the
-    # eight kernels a launch list of one decode step shows.
-    assert bench.launches_per_step(synth.WORKLOADS["step3_decode"]) == 8
-    assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 10
+    # router, top-k; the permutation (1 kernel up to 1024 rows, 3 above); the gather or
+    # FP8 quantisation; two GEMMs; the combine (the router weights' split is made once
+    # with the weights, not per step)
+    assert bench.launches_per_step(synth.WORKLOADS["step3_decode"]) == 7
+    assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 9
 
 
 def test_step_spread():
@@ -71,4 +71,38 @@ def test_design_bytes():
     assert a["design_bytes"] == 2 * R * per_row       # about 3.5 GB
     w = synth.WORKLOADS["step3_decode"]
     a = bench.algorithmic(w, w.T, np.arange(0, 49 * 16, 16), w.k)
-    assert a["design_bytes"] == 2 * (768 + 256) * (7168 * 2 + 5120 * 2 + 7168 * 4)
+    assert a["design_bytes"] == 2 * (768 + 256) * (7168 * 2 + 5120 * 4 + 7168 * 4)
+
+
+def test_expert_load_summary():
+    offsets = np.array([0, 5, 5, 12, 12, 20])          # 4 experts: 5, 0, 7, 0, 8 -> E = 5
+    e = bench.expert_load(offsets)
+    assert e["touched"] == 3 and e["pairs"] == 20 and e["max_rows"] == 8
+    assert e["min_rows_touched"] == 5 and abs(e["mean_rows_touched"] - 20 / 3) < 1e-12
+    assert bench.expert_load(np.zeros(4, dtype=int)) == {"touched": 0}
+
+
+def test_oracle_sample_spreads_over_the_batch():
+    idx = np.arange(100, 200)
+    s = bench.oracle_sample(idx, 5)
+    assert list(s) == [100, 125, 150, 174, 199] or list(s) == [100, 125, 150, 175, 199]
+    assert list(bench.oracle_sample(idx, 500)) == list(idx)
+
+
+def test_tp_check_rules():
+    import torch
+    ref = torch.randn(6, 32).to(torch.bfloat16)
+    valid = torch.tensor([1, 1, 1, 1, 0, 0], dtype=torch.uint8)
+    ref[4:] = 0
+    out = ref.clone()
+    assert bench.tp_check(out, ref, valid, 1, False)["ok"]
+    out[0, 0] = out[0, 0] + 0.5                        # any difference fails on one rank
+    assert not bench.tp_check(out, ref, valid, 1, False)["ok"]
+    r = bench.tp_check(out, ref, valid, 2, False)       # several ranks: the rms rule
+    assert r["max_err_over_rms"] > 0 and r["ok"] == (r["max_err_over_rms"] <= 2e-2)
+    small = ref.clone()
+    small[1, 1] = (small[1, 1].float() * (1 + 2 ** -7)).to(torch.bfloat16)
+    assert bench.tp_check(small, ref, valid, 2, False)["ok"]
+    bad_pad = ref.clone()
+    bad_pad[5, 3] = 1.0                                 # a padding row must stay +0.0
+    assert not bench.tp_check(bad_pad, ref, valid, 2, False)["ok"]

@@ -58,7 +58,7 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("WORLD_SIZE", "2")
     args = bench.argparse.Namespace(workload="step3_decode", steps=1, warmup=0, cpu_seconds=1.0,
-                                    experts=0)
+                                    reference_seconds=5.0, experts=0)
     assert bench.run_reference(args) is None
 
 
@@ -83,14 +83,33 @@ def test_reference_arm_line(capsys, monkeypatch):
     import oracle
     monkeypatch.setenv("RANK", "0")
     monkeypatch.setenv("WORLD_SIZE", "1")
-    args = bench.argparse.Namespace(workload="tiny", steps=2, warmup=0, cpu_seconds=0.2,
-                                    experts=0)
+    args = bench.argparse.Namespace(workload="tiny", steps=2, warmup=1, cpu_seconds=0.2,
+                                    reference_seconds=1.0, experts=0)
     res = bench.run_reference(args)
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line == json.loads(json.dumps(res))
     assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"]
     assert line["config"]["workload"] == "tiny" and line["n_gpus"] == 1
-    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["warmup"] == 1
     assert line["cpu_baseline"]["cores"] == oracle.max_threads() >= 1
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.parametrize("env,argv,want", [
+    ({"WORLD_SIZE": "1"}, [], ("native", "step3_decode", False)),
+    ({"WORLD_SIZE": "1"}, ["--workload", "fp8_prefill"], ("native", "fp8_prefill", True)),
+    ({"WORLD_SIZE": "2"}, [], ("tp", "step3_decode", False)),       # the scaling command
+    ({"WORLD_SIZE": "2"}, ["--replicas"], ("native", "step3_decode", False)),
+    ({"WORLD_SIZE": "1"}, ["--tp"], ("tp", "dp_padded", False)),
+    ({"WORLD_SIZE": "1"}, ["--impl", "reference"], ("reference", "step3_decode", False)),
+])
+def test_dispatch(monkeypatch, env, argv, want):
+    for kk, v in env.items():
+        monkeypatch.setenv(kk, v)
+    seen = []
+    for arm in ("native", "tp", "reference"):
+        monkeypatch.setattr(bench, f"run_{arm}",
+                            lambda a, arm=arm: seen.append((arm, a.workload, a.single)))
+    bench.main(argv)
+    assert seen == [want]
