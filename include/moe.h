@@ -71,6 +71,7 @@ typedef enum {
 #define MOE_DEV_WAIT_TIMEOUT_DOWN    0x2u   /* a bounded wait expired in the down GEMM */
 #define MOE_DEV_BAD_EXPERT_ID        0x4u   /* a routed expert index outside [0, E) */
 #define MOE_DEV_WAIT_TIMEOUT_ROUTER  0x8u   /* a bounded wait expired in the router GEMM */
+#define MOE_DEV_WAIT_TIMEOUT_SEND    0x10u  /* a sender gave up waiting for a group's tiles */
 
 /* Shape of the layer; fixed for the lifetime of a plan. */
 typedef struct {
@@ -225,6 +226,45 @@ moe_status moe_forward_scatter_experts(moe_plan_t plan, const moe_weights *weigh
                                        int expert_begin, int expert_end, void *workspace,
                                        size_t ws_bytes, void *stream, moe_debug *dbg);
 
+/* Expert-parallel rank with the per-pair return, sends overlapping the down GEMM
+ * ([SGLang] MoE 모델을 위한 Single Batch Overlap 기법, §핵심 코드 분석: a per-expert
+ * completion signal between the down projection GEMM and the combine's sends, and
+ * a set number of SMs for the sends).
+ *
+ * moe_forward_scatter_pairs computes, like moe_forward_scatter_experts, the
+ * routed experts [expert_begin, expert_end) of the plan (their weights given) for
+ * the gathered rows, but instead of a combine it returns every routed pair's
+ * expert output row unweighted, so each owner can sum a token's k rows in the
+ * one-GPU order.  The down GEMM's launch is cooperative: send_ctas of its CTAs
+ * (1 .. SMs - 1) do no tiles; each waits on a per-group counter that the other
+ * CTAs' epilogue warps raise after storing each tile, and as soon as an expert's
+ * tiles are all stored, copies its rows to the owners' slabs while later experts
+ * are still being multiplied.  The receive slab of owner r is fp32
+ * [n_slots][rows_per_rank][H], slot-major:
+ *   pair (t, j) of a routed expert -> dst[t / rows_per_rank] + (j * rows_per_rank
+ *                                     + t % rows_per_rank) * H,          j < k
+ *   the shared expert's row of t   -> slot shared_slot (>= k) likewise (plans with
+ *                                     num_shared = 1 only; ignored otherwise).
+ * dst: n_dst (1..8) device pointers, 16-byte aligned, possibly peer memory (the
+ * kernel only stores to them); n_dst * rows_per_rank == T.  Nothing but those
+ * rows is written to the slabs.  A sender that waits longer than the plan's wait
+ * limit sets MOE_DEV_WAIT_TIMEOUT_SEND and stops (its rows stay unsent).
+ *
+ * moe_reduce_pairs is the owner's half: out[t] = bf16(sum_{j<k} w[t,j] *
+ * slab[j][t] (fused multiply-adds, j ascending) + sum_{s<n_extra} slab[k+s][t]
+ * (s ascending)), padding rows +0.0; slab fp32 [k + n_extra][rows][H], w fp32
+ * [rows, k] (this owner's rows' routing weights), valid uint8 [rows] or NULL,
+ * out bf16 [rows, H]; H a multiple of 8, slab and out 16-byte aligned.  On one
+ * rank with every expert local this is the plain forward's combine, bit for bit. */
+moe_status moe_forward_scatter_pairs(moe_plan_t plan, const moe_weights *weights,
+                                     const void *hidden, const uint8_t *valid, int T, int k,
+                                     float *const *dst, int n_dst, int rows_per_rank,
+                                     int shared_slot, int expert_begin, int expert_end,
+                                     int send_ctas, void *workspace, size_t ws_bytes,
+                                     void *stream, moe_debug *dbg);
+moe_status moe_reduce_pairs(const float *slab, int k, int n_extra, int rows, int H,
+                            const float *w, const uint8_t *valid, void *out, void *stream);
+
 /* Routing only, from given fp32 logits [T, E] (device): the top-k selection,
  * weights, per-expert offsets and permutation exactly as moe_forward computes
  * them.  Outputs as in moe_debug (topk_ids, topk_w [T,k]; perm [T*k];
@@ -280,7 +320,9 @@ moe_status moe_check_device_status(moe_plan_t plan, void *workspace, void *strea
  * inspection after a forward (host arithmetic only; nothing is launched):
  *  row_token  int32 [R]     token index of each permuted row (R = Tv*(k+S))
  *  x_perm     [R, H]        permuted activations (bf16; e4m3 codes for FP8)
- *  h          [R, Imax]     SwiGLU output rows (bf16; e4m3 codes for FP8)
+ *  h          SwiGLU output rows: bf16 weights: [2R, Imax], row 2r = bf16(h_r) and
+ *                           row 2r + 1 = bf16(h_r - that) (two parts, multiplied both
+ *                           by the down GEMM); FP8: [R, Imax] e4m3 codes
  *  y          [R, H]        expert output rows before the weighted combine
  *                           (fp32 for bf16 weights, bf16 for FP8 weights)
  *  group_offsets int32 [E+S+1]: rows of expert e are [go[e], go[e+1]); the

@@ -27,6 +27,7 @@ MOE_DEV_WAIT_TIMEOUT_GATE_UP = 0x1
 MOE_DEV_WAIT_TIMEOUT_DOWN = 0x2
 MOE_DEV_BAD_EXPERT_ID = 0x4
 MOE_DEV_WAIT_TIMEOUT_ROUTER = 0x8
+MOE_DEV_WAIT_TIMEOUT_SEND = 0x10
 
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "permute", "gather", "gate_up_gemm", "down_gemm", "combine")
@@ -37,7 +38,8 @@ EXPORTED = ("moe_plan_create", "moe_plan_destroy", "moe_plan_set_wait_limit", "m
             "moe_get_workspace_views", "moe_status_string", "moe_last_cuda_error_string",
             "moe_pipeline_slot_bytes", "moe_pipeline_create", "moe_pipeline_submit",
             "moe_pipeline_synchronize", "moe_pipeline_streams", "moe_pipeline_destroy",
-            "moe_router_split_bytes", "moe_split_router_weights")
+            "moe_router_split_bytes", "moe_split_router_weights", "moe_forward_scatter_pairs",
+            "moe_reduce_pairs")
 MAX_TP_RANKS = 8
 
 MOE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -135,6 +137,12 @@ def load():
     L.moe_pipeline_streams.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                        ctypes.POINTER(_vp)]
     L.moe_pipeline_streams.restype = _c_int
+    L.moe_forward_scatter_pairs.argtypes = [_vp, ctypes.POINTER(moe_weights), _vp, _vp, _c_int,
+                                            _c_int, _vp, _c_int, _c_int, _c_int, _c_int,
+                                            _c_int, _c_int, _vp, ctypes.c_size_t, _vp, _vp]
+    L.moe_forward_scatter_pairs.restype = _c_int
+    L.moe_reduce_pairs.argtypes = [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]
+    L.moe_reduce_pairs.restype = _c_int
     L.moe_router_split_bytes.argtypes = [_vp]
     L.moe_router_split_bytes.restype = ctypes.c_size_t
     L.moe_split_router_weights.argtypes = [_vp, _vp, _vp, ctypes.c_size_t, _vp]
@@ -279,6 +287,30 @@ def moe_forward_scatter_experts(plan, weights: moe_weights, hidden, valid, T: in
                                             ws_bytes, _stream(stream),
                                             None if dbg is None else ctypes.byref(dbg))
     _check(st, "moe_forward_scatter_experts")
+
+
+def moe_forward_scatter_pairs(plan, weights: moe_weights, hidden, valid, T: int, k: int, dst,
+                              rows_per_rank: int, shared_slot: int, expert_begin: int,
+                              expert_end: int, send_ctas: int, workspace, ws_bytes: int,
+                              stream=None, dbg: moe_debug | None = None) -> None:
+    """dst: the owners' per-pair receive slabs (device addresses or tensors)."""
+    arr = (_vp * len(dst))(*[_addr(d, "dst", _F32) for d in dst])
+    st = load().moe_forward_scatter_pairs(plan, ctypes.byref(weights),
+                                          _addr(hidden, "hidden", _BF16),
+                                          _addr(valid, "valid", _MASK), T, k, arr, len(dst),
+                                          rows_per_rank, shared_slot, expert_begin, expert_end,
+                                          send_ctas, _addr(workspace, "workspace"), ws_bytes,
+                                          _stream(stream),
+                                          None if dbg is None else ctypes.byref(dbg))
+    _check(st, "moe_forward_scatter_pairs")
+
+
+def moe_reduce_pairs(slab, k: int, n_extra: int, rows: int, H: int, w, valid, out,
+                     stream=None) -> None:
+    st = load().moe_reduce_pairs(_addr(slab, "slab", _F32), k, n_extra, rows, H,
+                                 _addr(w, "w", _F32), _addr(valid, "valid", _MASK),
+                                 _addr(out, "out", _BF16), _stream(stream))
+    _check(st, "moe_reduce_pairs")
 
 
 def moe_reduce_partials(slots, n_slots: int, rows: int, H: int, valid, out, stream=None) -> None:
@@ -479,6 +511,18 @@ class Plan:
         moe_forward_scatter_experts(self.handle, weights, hidden, valid, T, k, dst,
                                     rows_per_rank, slot, expert_begin, expert_end,
                                     self.workspace, self.ws_bytes, stream, dbg)
+
+    def forward_scatter_pairs(self, weights: moe_weights, hidden, valid, k: int, dst,
+                              rows_per_rank: int, shared_slot: int, expert_begin: int,
+                              expert_end: int, send_ctas: int, stream=None, dbg=None):
+        T = self._rows(hidden, valid)
+        need = (k + 1) * rows_per_rank * self.cfg.hidden
+        for d in dst:
+            if not isinstance(d, int) and d.numel() < need:
+                raise ValueError(f"dst: a slab of {d.numel()} values, needs at least {need}")
+        moe_forward_scatter_pairs(self.handle, weights, hidden, valid, T, k, dst, rows_per_rank,
+                                  shared_slot, expert_begin, expert_end, send_ctas,
+                                  self.workspace, self.ws_bytes, stream, dbg)
 
     def route_from_logits(self, logits, valid, k: int, topk_ids, topk_w, perm, offsets,
                           stream=None):

@@ -10,6 +10,15 @@
 //                                              u = Wu[e][i,:] . x_perm[r,:]
 //   down:             y[r, o] = Wd[e][o,:] . h[r,:]     (kept in fp32 for the combine)
 //
+// h leaves the gated epilogue in two bf16 parts, hi = bf16(h) and lo = bf16(h - hi),
+// stored as rows 2r and 2r + 1 of the h buffer, and the down GEMM multiplies both
+// (2N rows on the MMA's N side) and adds the two columns of a row in fp32: the
+// tensor core takes bf16 operands, and the two parts carry h to 16 significant
+// bits instead of 8, so rounding h no longer shows in the layer's output (with
+// hi alone it cost up to about half a percent of the output rms, which with the
+// output's own bf16 rounding came close to the 2 % bound).  The down GEMM takes
+// at most 96 rows a tile, so that a tile's 2 x 96 part rows fit one 192-row box.
+//
 // for every permuted row r of group e (routed experts, then the shared one).
 // Decode batches give each expert only a handful of rows, so the weights take
 // the MMA's M side (128 weight rows per tile) and the rows take N (16..128,
@@ -24,6 +33,12 @@
 // overlap the main loop of the next.  Tiles are enumerated on the device from
 // the group offsets (no host round trip), and every CTA walks tiles
 // blockIdx.x, blockIdx.x + gridDim.x, ...  Every wait is bounded.
+//
+// Signalled sends (down GEMM of an expert-parallel rank): the launch is
+// cooperative (all CTAs resident), its first n_gemm CTAs run the tiles as above
+// and every epilogue warp counts each stored tile in its group's counter; the
+// other CTAs copy each group's rows to the owners' slabs as soon as the group's
+// count is complete, while later groups are still being multiplied.
 #include <cudaTypedefs.h>
 
 #include "moe_internal.cuh"
@@ -33,7 +48,10 @@ namespace {
 
 constexpr int BM = 128;            // weight rows per MMA
 constexpr int BK = 64;             // K elements per stage (128 bytes of bf16: one swizzle row)
-constexpr int BN = 128;            // max activation rows per tile
+constexpr int BN = 128;            // max activation rows per gated tile
+constexpr int BN_DOWN = 96;        // max h rows per down tile: 2 x 96 part rows per box
+template <bool GATED>
+__host__ __device__ constexpr int tile_rows() { return GATED ? BN : BN_DOWN; }
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccStride = 256;    // TMEM columns between the two accumulator buffers
@@ -42,10 +60,12 @@ constexpr unsigned long long kTeardownLimitNs = 1000000000ull;
 template <bool GATED>
 struct Cfg {
   static constexpr int A_BYTES = (GATED ? 2 : 1) * BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
-  // down: one weight box per stage, so more stages keep enough HBM bytes in flight
-  // (7 x 32 KB + 3 KB fills the 227 KB a CTA may have)
-  static constexpr int STAGES = GATED ? 4 : 7;
+  // the largest B box: 128 activation rows (gated) or 2 x 96 part rows of h (down)
+  static constexpr int B_ROWS = GATED ? BN : 2 * BN_DOWN;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  // down: one weight box per stage, so more stages keep HBM bytes in flight
+  // (5 x 40 KB + 3 KB of the 227 KB a CTA may have)
+  static constexpr int STAGES = GATED ? 4 : 5;
   static constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
   static constexpr int SMEM_BYTES = DATA_BYTES + 1024 + 2048;
 };
@@ -63,13 +83,17 @@ struct KParams {
   unsigned int* status;
   unsigned int timeout_bit;
   unsigned long long wait_limit_ns;
+  int n_gemm;       // CTAs that run tiles (the rest send)
+  SendArgs send;
 };
 
 struct Tile {
   int g, m, row0, nrows, n_mma, k_blocks;
 };
 
+template <bool GATED>
 __device__ __forceinline__ Tile decode_tile(int t, const int* ts, const int* go, const KParams& p) {
+  constexpr int TR = tile_rows<GATED>();
   int lo = 0, hi = p.G;   // invariant: ts[lo] <= t < ts[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -78,12 +102,12 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* ts, const int* go,
   Tile ti;
   ti.g = lo;
   const int gbeg = go[lo], gend = go[lo + 1];
-  const int nt = (gend - gbeg + BN - 1) / BN;
+  const int nt = (gend - gbeg + TR - 1) / TR;
   const int local = t - ts[lo];
   ti.m = local / nt;
   const int n = local - ti.m * nt;
-  ti.row0 = gbeg + n * BN;
-  ti.nrows = min(BN, gend - ti.row0);
+  ti.row0 = gbeg + n * TR;
+  ti.nrows = min(TR, gend - ti.row0);
   ti.n_mma = (ti.nrows + 15) & ~15;
   ti.k_blocks = lo < p.E ? p.kb_routed : p.kb_shared;
   return ti;
@@ -114,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* go = p.group_offsets;
+  const bool sender = !GATED && p.send.n_send > 0 && (int)blockIdx.x >= p.n_gemm;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -133,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmB64);
     tma_prefetch_desc(&tmB128);
   }
-  if (warp == 1) {
+  if (warp == 1 && !sender) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
@@ -145,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int cnt = 0;
       if (g < p.G) {
         const int rows = go[g + 1] - go[g];
-        cnt = (g < p.E ? p.m_routed : p.m_shared) * ((rows + BN - 1) / BN);
+        cnt = (g < p.E ? p.m_routed : p.m_shared) *
+              ((rows + tile_rows<GATED>() - 1) / tile_rows<GATED>());
       }
       int incl = cnt;
 #pragma unroll
@@ -161,8 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
   const int total = ts[p.G];
+  if (sender) {
+    // 4 epilogue warps count every tile
+    send_finished_groups<float>(p.send, static_cast<const float*>(p.d), p.ldd, go, ts, p.G, p.E,
+                                4u, (int)blockIdx.x - p.n_gemm, p.status, p.wait_limit_ns,
+                                reinterpret_cast<int*>(tmem_holder));
+    return;
+  }
+  const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -172,17 +205,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, parity = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile ti = decode_tile(t, ts, go, p);
+      for (int t = blockIdx.x; t < total && ok; t += p.n_gemm) {
+        const Tile ti = decode_tile<GATED>(t, ts, go, p);
         const bool routed = ti.g < p.E;
         const CUtensorMap* am = routed ? &tmA : &tmAs;
         const int arow = (routed ? (ti.g - p.e_base) * p.rows_per_expert : 0) + ti.m * BM;
         const int up = routed ? p.up_routed : p.up_shared;
         // the tile's rows in one box of 16/32/64/128 rows (one copy from the single
-        // producer thread per K block; rows past the group come from L2 and go unused)
-        const int box = ti.n_mma <= 16 ? 16 : ti.n_mma <= 32 ? 32 : ti.n_mma <= 64 ? 64 : 128;
+        // producer thread per K block; rows past the group come from L2 and go unused);
+        // down: the h rows' two parts, 2 x n_mma rows from row 2 x row0
+        // (box heights: gated 16/32/64/128, down 32/64/128/192 part rows)
+        const int brows = GATED ? ti.n_mma : 2 * ti.n_mma;
+        const int b0 = GATED ? 16 : 32;
+        const int box = brows <= b0 ? b0 : brows <= 2 * b0 ? 2 * b0 : brows <= 4 * b0 ? 4 * b0
+                      : C::B_ROWS;
         const CUtensorMap* bm =
-            box == 16 ? &tmB16 : box == 32 ? &tmB32 : box == 64 ? &tmB64 : &tmB128;
+            box == b0 ? &tmB16 : box == 2 * b0 ? &tmB32 : box == 4 * b0 ? &tmB64 : &tmB128;
         const uint32_t bytes = C::A_BYTES + box * BK * 2;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, p.wait_limit_ns, p.status,
@@ -196,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(a_dst, am, kb * BK, arow, fb, pol_a);
           if (GATED) tma_load_2d(a_dst + BM * BK * 2, am, kb * BK, arow + up, fb, pol_a);
           const uint32_t b_dst = smem_u32(b_smem + stage * C::B_BYTES);
-          tma_load_2d(b_dst, bm, kb * BK, ti.row0, fb, pol_b);
+          tma_load_2d(b_dst, bm, kb * BK, GATED ? ti.row0 : 2 * ti.row0, fb, pol_b);
           issued |= 1u << stage;
           parity = (parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -216,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       bool ok = true, any = false;
       int local = 0;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++local) {
-        const Tile ti = decode_tile(t, ts, go, p);
+      for (int t = blockIdx.x; t < total && ok; t += p.n_gemm, ++local) {
+        const Tile ti = decode_tile<GATED>(t, ts, go, p);
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
         if (!mbar_wait_bounded(smem_u32(&tempty[buf]), (use & 1u) ^ 1u, p.wait_limit_ns, p.status,
@@ -226,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_m128(ti.n_mma);
+        const uint32_t idesc = idesc_bf16_m128(GATED ? ti.n_mma : 2 * ti.n_mma);
         const uint32_t d_gate = tmem_base + buf * kAccStride;
         const uint32_t d_up = d_gate + BN;
         for (int kb = 0; kb < ti.k_blocks; ++kb) {
@@ -265,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------------- epilogue
     const int q = warp & 3;               // TMEM lane quadrant of this warp
     int local = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
-      const Tile ti = decode_tile(t, ts, go, p);
+    for (int t = blockIdx.x; t < total; t += p.n_gemm, ++local) {
+      const Tile ti = decode_tile<GATED>(t, ts, go, p);
       const int buf = local & 1;
       const uint32_t use = (uint32_t)(local >> 1);
       if (!mbar_wait_bounded_warp(smem_u32(&tfull[buf]), use & 1u, p.wait_limit_ns, p.status,
@@ -276,29 +314,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kAccStride;
       const int col = ti.m * BM + q * 32 + lane;
       const size_t dofs = (size_t)ti.row0 * p.ldd + col;
-      for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-        float g[16];
-        tmem_ld_16(tbase + c0, g);
-        if (GATED) {
-          float u[16];
+      if (GATED) {
+        // h = silu(g) * u as two bf16 parts: hi in row 2r, lo = bf16(h - hi) in row 2r + 1
+        __nv_bfloat16* h2 = static_cast<__nv_bfloat16*>(p.d) + (size_t)2 * ti.row0 * p.ldd + col;
+        for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+          float g[16], u[16];
+          tmem_ld_16(tbase + c0, g);
           tmem_ld_16(tbase + BN + c0, u);
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             if (c0 + c < ti.nrows) {
-              const float s = g[c] / (1.0f + __expf(-g[c]));
-              static_cast<__nv_bfloat16*>(p.d)[dofs + (size_t)(c0 + c) * p.ldd] =
-                  __float2bfloat16_rn(s * u[c]);
+              const float h = g[c] / (1.0f + __expf(-g[c])) * u[c];
+              const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+              h2[(size_t)(2 * (c0 + c)) * p.ldd] = hi;
+              h2[(size_t)(2 * (c0 + c) + 1) * p.ldd] = lo;
             }
           }
-        } else {
+        }
+      } else {
+        // columns 2c and 2c + 1 are row c's products with hi and lo
+        for (int c0 = 0; c0 < 2 * ti.n_mma; c0 += 16) {
+          float v[16];
+          tmem_ld_16(tbase + c0, v);
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            if (c0 + c < ti.nrows) static_cast<float*>(p.d)[dofs + (size_t)(c0 + c) * p.ldd] = g[c];
+          for (int c = 0; c < 8; ++c) {
+            const int r = c0 / 2 + c;
+            if (r < ti.nrows)
+              static_cast<float*>(p.d)[dofs + (size_t)r * p.ldd] = v[2 * c] + v[2 * c + 1];
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+      if (!GATED && p.send.n_send > 0) signal_tile_stored(p.send.done, ti.g);
     }
   }
 
@@ -362,10 +412,15 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   } else {
     tmAs = tmA;
   }
-  if (!make_map_bf16(&tmB16, a.b, a.K_ld, (uint64_t)a.R_cap, 16) ||
-      !make_map_bf16(&tmB32, a.b, a.K_ld, (uint64_t)a.R_cap, 32) ||
-      !make_map_bf16(&tmB64, a.b, a.K_ld, (uint64_t)a.R_cap, 64) ||
-      !make_map_bf16(&tmB128, a.b, a.K_ld, (uint64_t)a.R_cap, 128))
+  // down: the h buffer holds two bf16 parts (rows 2r, 2r + 1) for each of R_cap rows,
+  // read in boxes of 32/64/128/192 part rows (gated: 16/32/64/128 rows)
+  const uint64_t b_rows = (uint64_t)a.R_cap * (a.gated ? 1 : 2);
+  const uint32_t b0 = a.gated ? 16 : 32;
+  const uint32_t b3 = a.gated ? Cfg<true>::B_ROWS : Cfg<false>::B_ROWS;
+  if (!make_map_bf16(&tmB16, a.b, a.K_ld, b_rows, b0) ||
+      !make_map_bf16(&tmB32, a.b, a.K_ld, b_rows, 2 * b0) ||
+      !make_map_bf16(&tmB64, a.b, a.K_ld, b_rows, 4 * b0) ||
+      !make_map_bf16(&tmB128, a.b, a.K_ld, b_rows, b3))
     return cudaErrorInvalidValue;
 
   KParams p;
@@ -385,12 +440,30 @@ cudaError_t launch_grouped_gemm(const GroupedGemmArgs& a, cudaStream_t st) {
   p.status = a.status;
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.send = a.send;
+  if (a.gated) p.send.n_send = 0;
+  p.n_gemm = a.num_ctas - p.send.n_send;
+  if (p.n_gemm < 1) return cudaErrorInvalidValue;
   if (a.gated) {
     grouped_gemm_kernel<true><<<a.num_ctas, kThreads, Cfg<true>::SMEM_BYTES, st>>>(
         tmA, tmAs, tmB16, tmB32, tmB64, tmB128, p);
-  } else {
+  } else if (p.send.n_send == 0) {
     grouped_gemm_kernel<false><<<a.num_ctas, kThreads, Cfg<false>::SMEM_BYTES, st>>>(
         tmA, tmAs, tmB16, tmB32, tmB64, tmB128, p);
+  } else {
+    // the senders wait on the tiles: every CTA must be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_ctas, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg<false>::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<false>, tmA, tmAs, tmB16, tmB32, tmB64,
+                              tmB128, p);
   }
   return cudaGetLastError();
 }

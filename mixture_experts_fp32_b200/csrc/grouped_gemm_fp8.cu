@@ -39,6 +39,11 @@
 //   down:  a tile owns up to 256 output features (two weight scale blocks); y
 //          is written in bf16.
 //
+// Signalled sends (down GEMM of an expert-parallel rank): a cooperative launch
+// whose first n_gemm CTAs run the tiles, every epilogue warp counting each stored
+// tile in its group's counter, while the other CTAs copy each finished group's
+// rows to the owners' slabs.
+//
 // Three warpgroups (384 threads).  Warpgroup 0: warp 0 issues TMA loads, warp 1
 // owns tensor memory and issues the MMAs; it gives registers back
 // (setmaxnreg.dec).  Warpgroups 1 and 2 (8 warps) promote and finish, with the
@@ -141,6 +146,8 @@ struct KParams8 {
   unsigned int* status;
   unsigned int timeout_bit;
   unsigned long long wait_limit_ns;
+  int n_gemm;                     // CTAs that run tiles (the rest send)
+  SendArgs send;
 };
 
 struct Tile8 {
@@ -204,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* go = gos;
-  const int cta = blockIdx.x, nctas = gridDim.x;
+  const int cta = blockIdx.x, nctas = p.n_gemm;
+  const bool sender = !GATED && p.send.n_send > 0 && cta >= p.n_gemm;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -221,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmWs);
   }
-  if (warp == 1) {
+  if (warp == 1 && !sender) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
     tmem_relinquish();
   }
@@ -254,8 +262,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
   const int total = ts[p.G];
+  if (sender) {
+    // 8 epilogue warps count every tile; y rows are bf16
+    send_finished_groups<__nv_bfloat16>(p.send, static_cast<const __nv_bfloat16*>(p.d), p.ldd,
+                                        go, ts, p.G, p.E, (unsigned int)kEpiWarps,
+                                        cta - p.n_gemm, p.status, p.wait_limit_ns,
+                                        reinterpret_cast<int*>(tmem_holder));
+    return;
+  }
+  const uint32_t tmem_base = *tmem_holder;
 
   if (warp < 4) {
     regs_dec<kProducerRegs>();
@@ -356,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // scales requested) before the current tile's finishing work, so that the
     // loads' latency hides behind it.
     struct EpiTile {
-      int row0, rows, f0, nfeat, k_blocks;
+      int g, row0, rows, f0, nfeat, k_blocks;
       const float* sa_row;
       const float* swa;
       const float* swb;
@@ -364,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto setup = [&](int t, EpiTile& e, float& a0, float& wa0, float& wb0) {
       const Tile8 ti = decode_tile8<GATED>(t, ts, go, p);
       const bool routed = ti.g < p.E;
+      e.g = ti.g;
       e.row0 = ti.row0;
       e.rows = ti.nrows;
       e.f0 = ti.f0;
@@ -508,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[w8] = o;
         }
       }
+      if (!GATED && p.send.n_send > 0) signal_tile_stored(p.send.done, fin.g);
     }
   }
 
@@ -609,11 +627,29 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   p.status = a.status;
   p.timeout_bit = a.timeout_bit;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.send = a.send;
+  if (a.gated) p.send.n_send = 0;
+  p.n_gemm = a.num_ctas - p.send.n_send;
+  if (p.n_gemm < 1) return cudaErrorInvalidValue;
 
-  if (a.gated)
+  if (a.gated) {
     grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
-  else
+  } else if (p.send.n_send == 0) {
     grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
+  } else {
+    // the senders wait on the tiles: every CTA must be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_ctas, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_fp8_kernel<false>, tmA, tmW, tmWs, p);
+  }
   return cudaGetLastError();
 }
 

@@ -17,8 +17,8 @@ struct moe_plan_s {
   int ks_max;        // top_k_max + S
   size_t r_cap;      // max_tokens * ks_max rows
   // byte offsets inside the workspace
-  size_t off_status, off_goff, off_wsplit, off_rscratch, off_partial, off_logits, off_ids, off_w,
-      off_perm,
+  size_t off_status, off_goff, off_done, off_wsplit, off_rscratch, off_partial, off_logits,
+      off_ids, off_w, off_perm,
       off_inv, off_rowtok, off_xp, off_sx, off_h, off_sh, off_y;
   unsigned long long wait_limit_ns;
   int device;
@@ -142,6 +142,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   };
   p->off_status = take(64);
   p->off_goff = take(sizeof(int) * (E + 2));
+  p->off_done = take(sizeof(unsigned int) * (E + 2));
   p->off_wsplit = take(2 * 3 * (size_t)moe::router_padded_experts((int)E) * H);
   p->off_rscratch = take(sizeof(int) * (size_t)moe::route_scratch_ints((int)T, (int)E));
   p->off_partial = take(sizeof(float) * moe::kRouterSplitMax * T * E);
@@ -152,10 +153,10 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   p->off_inv = take(sizeof(int) * T * ks);
   p->off_rowtok = take(sizeof(int) * r_cap);
   if (c.wtype == MOE_W_BF16) {
-    // bf16 permuted rows and h; fp32 expert outputs
+    // bf16 permuted rows; h as two bf16 parts a row (rows 2r, 2r + 1); fp32 expert outputs
     p->off_xp = take(2 * r_cap * H);
     p->off_sx = 0;
-    p->off_h = take(2 * r_cap * (size_t)imax);
+    p->off_h = take(2 * 2 * r_cap * (size_t)imax);
     p->off_sh = 0;
     p->off_y = take(sizeof(float) * r_cap * H);
   } else {
@@ -210,7 +211,7 @@ MOE_EXPORT moe_status moe_split_router_weights(moe_plan_t plan, const float* rou
 static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const void* hidden,
                                const uint8_t* valid, int T, int k, const moe::CombineOut& co,
                                int eb, int ee, void* workspace, size_t ws_bytes, void* stream,
-                               moe_debug* dbg) {
+                               moe_debug* dbg, const moe::SendArgs* send = nullptr) {
   moe_status s = check_common(plan, T, k, workspace, ws_bytes);
   if (s != MOE_OK) return s;
   if (wts == nullptr) return MOE_ERR_INVALID_ARG;
@@ -234,6 +235,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     return MOE_ERR_INVALID_ARG;
   s = ensure_device(plan);
   if (s != MOE_OK) return s;
+  if (send != nullptr && (send->n_send < 1 || send->n_send >= plan->num_sms))
+    return MOE_ERR_INVALID_ARG;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = c.num_experts, H = c.hidden, I = c.inter, Is = S ? c.shared_inter : 0;
@@ -338,11 +341,19 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     ga.ldd = H;
     ga.gated = false;
     ga.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
+    if (send != nullptr) {
+      ga.send = *send;
+      ga.send.perm = perm;
+      ga.send.row_token = rowtok;
+      ga.send.done = at<unsigned int>(workspace, plan->off_done);
+      if (cudaMemsetAsync(ga.send.done, 0, sizeof(unsigned int) * G, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     s = check_launch(moe::launch_grouped_gemm(ga, st));
     if (s != MOE_OK) return s;
     record(dbg, 6, st);
 
-    s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S, co, st));
+    if (send == nullptr) s = check_launch(moe::launch_combine(y, H, inv, w, valid, T, k, S, co, st));
   } else {
     moe::GroupedGemmFp8Args fa;
     memset(&fa, 0, sizeof(fa));
@@ -398,11 +409,20 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
     fa.ldd = H;
     fa.gated = false;
     fa.timeout_bit = MOE_DEV_WAIT_TIMEOUT_DOWN;
+    if (send != nullptr) {
+      fa.send = *send;
+      fa.send.perm = perm;
+      fa.send.row_token = rowtok;
+      fa.send.done = at<unsigned int>(workspace, plan->off_done);
+      if (cudaMemsetAsync(fa.send.done, 0, sizeof(unsigned int) * G, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
     s = check_launch(moe::launch_grouped_gemm_fp8(fa, st));
     if (s != MOE_OK) return s;
     record(dbg, 6, st);
 
-    s = check_launch(moe::launch_combine_bf16y(y16, H, inv, w, valid, T, k, S, co, st));
+    if (send == nullptr)
+      s = check_launch(moe::launch_combine_bf16y(y16, H, inv, w, valid, T, k, S, co, st));
   }
   if (s != MOE_OK) return s;
   record(dbg, 7, st);
@@ -476,6 +496,50 @@ MOE_EXPORT moe_status moe_reduce_partials(const float* slots, int n_slots, int r
     return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
   return check_launch(moe::launch_reduce_slots(slots, n_slots, rows, H, valid,
+                                               static_cast<__nv_bfloat16*>(out),
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+MOE_EXPORT moe_status moe_forward_scatter_pairs(moe_plan_t plan, const moe_weights* wts,
+                                                const void* hidden, const uint8_t* valid, int T,
+                                                int k, float* const* dst, int n_dst,
+                                                int rows_per_rank, int shared_slot,
+                                                int expert_begin, int expert_end, int send_ctas,
+                                                void* workspace, size_t ws_bytes, void* stream,
+                                                moe_debug* dbg) {
+  if (plan == nullptr || expert_begin < 0 || expert_end <= expert_begin ||
+      expert_end > plan->cfg.num_experts || send_ctas < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (dst == nullptr || n_dst < 1 || n_dst > moe::kMaxTpRanks || rows_per_rank < 1 ||
+      (long long)n_dst * rows_per_rank != T)
+    return MOE_ERR_INVALID_ARG;
+  if (plan->cfg.num_shared && shared_slot < k) return MOE_ERR_INVALID_ARG;
+  moe::SendArgs sa;
+  memset(&sa, 0, sizeof(sa));
+  for (int r = 0; r < n_dst; ++r) {
+    if (dst[r] == nullptr || !aligned16(dst[r])) return MOE_ERR_INVALID_ARG;
+    sa.dst[r] = dst[r];
+  }
+  sa.rows_per_rank = rows_per_rank;
+  sa.k = k;
+  sa.shared_slot = shared_slot;
+  sa.n_send = send_ctas;
+  sa.timeout_bit = MOE_DEV_WAIT_TIMEOUT_SEND;
+  moe::CombineOut co;
+  memset(&co, 0, sizeof(co));
+  return forward_impl(plan, wts, hidden, valid, T, k, co, expert_begin, expert_end, workspace,
+                      ws_bytes, stream, dbg, &sa);
+}
+
+MOE_EXPORT moe_status moe_reduce_pairs(const float* slab, int k, int n_extra, int rows, int H,
+                                       const float* w, const uint8_t* valid, void* out,
+                                       void* stream) {
+  if (slab == nullptr || w == nullptr || out == nullptr || k < 1 || k > moe::kMaxTopK ||
+      n_extra < 0 || n_extra > moe::kMaxTpRanks || rows < 0 || H <= 0 || H % 8 != 0 ||
+      !aligned16(slab) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  return check_launch(moe::launch_reduce_pairs(slab, k, n_extra, rows, H, w, valid,
                                                static_cast<__nv_bfloat16*>(out),
                                                static_cast<cudaStream_t>(stream)));
 }

@@ -27,6 +27,27 @@ struct CombineOut {
   int slot;
 };
 
+// The per-pair return of an expert-parallel rank (signalled sends overlapping
+// the down GEMM, [SGLang] MoE 모델을 위한 Single Batch Overlap 기법, §핵심 코드 분석):
+// the down GEMM's launch also holds `n_send` CTAs that wait on a per-group
+// completion counter (raised by every epilogue warp after it has stored a tile of
+// that group) and copy each finished group's expert-output rows, unweighted, into
+// the receive slab of the rank that owns the row's token:
+//   routed pair (t, j): dst[t / rows] + (j * rows + t % rows) * H
+//   shared row of t:    dst[t / rows] + (shared_slot * rows + t % rows) * H
+// as fp32 (widened from bf16 on the FP8 path).
+struct SendArgs {
+  float* dst[kMaxTpRanks];     // one receive slab per owning rank (may be peer memory)
+  int rows_per_rank;
+  int k;                       // routed slots per row in a slab
+  int shared_slot;             // slot of the shared expert's rows (k)
+  const int* perm;             // pair index t*k+j of each routed permuted row
+  const int* row_token;        // token of each permuted row
+  unsigned int* done;          // [G] completion counters, zeroed before the launch
+  int n_send;                  // CTAs of the launch that send (0: no sending)
+  unsigned int timeout_bit;
+};
+
 // ------------------------------------------------------------------ host side
 
 struct GroupedGemmArgs {
@@ -50,6 +71,7 @@ struct GroupedGemmArgs {
   unsigned int timeout_bit;
   unsigned long long wait_limit_ns;
   int num_ctas;
+  SendArgs send;               // down GEMM only: signalled sends (n_send > 0: cooperative)
 };
 
 // e4m3 grouped GEMM with one fp32 scale per 128x128 weight block and per 1x128
@@ -77,6 +99,7 @@ struct GroupedGemmFp8Args {
   unsigned int timeout_bit;
   unsigned long long wait_limit_ns;
   int num_ctas;
+  SendArgs send;               // down GEMM only: signalled sends (n_send > 0: cooperative)
 };
 
 // FP8: quantise every valid token once (1x128 groups) and store codes and scales into
@@ -119,6 +142,11 @@ cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w
 // out[t] = bf16(sum over slots g ascending of slots[g][t]); rows with valid[t] == 0 -> +0.0
 cudaError_t launch_reduce_slots(const float* slots, int n_slots, int rows, int H,
                                 const uint8_t* valid, __nv_bfloat16* out, cudaStream_t st);
+// Owner of a per-pair slab [k + n_extra][rows][H]: out[t] = bf16(sum_j w[t,j] * slab[j][t]
+// (fused multiply-adds, j ascending) + sum_s slab[k + s][t] (s ascending)); padding rows +0.0.
+cudaError_t launch_reduce_pairs(const float* slab, int k, int n_extra, int rows, int H,
+                                const float* w, const uint8_t* valid, __nv_bfloat16* out,
+                                cudaStream_t st);
 cudaError_t prepare_grouped_gemm_kernels();
 const moe_config* plan_config(const moe_plan_s* plan);
 void router_split_plan(int T, int E, int H, int num_sms, int* splits, int* kb_per_split);
@@ -445,6 +473,97 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 __device__ __forceinline__ uint32_t idesc_bf16_m128(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Raised by one lane of an epilogue warp once the warp's stores of a tile of
+// group g are done (the warp barrier orders the other lanes' stores before it;
+// the fence makes them visible device-wide before the count).
+__device__ __forceinline__ void signal_tile_stored(unsigned int* done, int g) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    __threadfence();
+    atomicAdd(done + g, 1u);
+  }
+}
+
+// The send role of a down-GEMM launch with signalled sends: CTA `sid` of `n_send`
+// walks the groups in the GEMM's tile order, waits (one thread, bounded) until the
+// group's counter reaches `per_tile` x its tile count, then its warps copy their
+// share of the group's rows into the owners' slabs.  After an expired wait it
+// sets the status bit and stops.  YT: the row type of y (fp32, or bf16 widened).
+template <typename YT>
+__device__ void send_finished_groups(const SendArgs& sa, const YT* __restrict__ y, int H,
+                                     const int* go, const int* ts, int G, int E,
+                                     unsigned int per_tile, int sid, unsigned int* status,
+                                     unsigned long long limit_ns, int* flag_smem) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int stride = sa.n_send * nwarps;
+  for (int g = 0; g < G; ++g) {
+    const int beg = go[g], rows = go[g + 1] - beg;
+    if (rows == 0) continue;
+    if (threadIdx.x == 0) {
+      const unsigned int target = per_tile * (unsigned int)(ts[g + 1] - ts[g]);
+      int ok = ld_acquire_gpu(sa.done + g) >= target;
+      if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        while (!(ok = ld_acquire_gpu(sa.done + g) >= target)) {
+          if (global_timer_ns() - t0 >= limit_ns) break;
+          __nanosleep(256);
+        }
+      }
+      if (!ok) atomicOr(status, sa.timeout_bit);
+      *flag_smem = ok;
+    }
+    __syncthreads();
+    const int ok = *flag_smem;
+    __syncthreads();
+    if (!ok) return;
+    for (int i = sid * nwarps + warp; i < rows; i += stride) {
+      const int pr = beg + i;
+      int t, slot;
+      if (g < E) {
+        const int pair = sa.perm[pr];
+        t = pair / sa.k;
+        slot = pair - t * sa.k;
+      } else {
+        t = sa.row_token[pr];
+        slot = sa.shared_slot;
+      }
+      const int owner = t / sa.rows_per_rank, lt = t - owner * sa.rows_per_rank;
+      float* base = sa.dst[0];
+#pragma unroll
+      for (int r = 1; r < kMaxTpRanks; ++r)
+        if (owner == r) base = sa.dst[r];
+      float4* dst = reinterpret_cast<float4*>(base + ((size_t)slot * sa.rows_per_rank + lt) * H);
+      const YT* src = y + (size_t)pr * H;
+      for (int v = lane; v < H / 8; v += 32) {
+        float f[8];
+        if constexpr (sizeof(YT) == 4) {
+          const float4 a = reinterpret_cast<const float4*>(src)[2 * v];
+          const float4 b = reinterpret_cast<const float4*>(src)[2 * v + 1];
+          f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+          f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        } else {
+          const uint4 r = reinterpret_cast<const uint4*>(src)[v];
+          const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            f[2 * q] = __uint_as_float(wv[q] << 16);               // bf16 -> fp32, exact
+            f[2 * q + 1] = __uint_as_float(wv[q] & 0xffff0000u);
+          }
+        }
+        dst[2 * v] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[2 * v + 1] = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+  }
 }
 
 #endif  // __CUDACC__

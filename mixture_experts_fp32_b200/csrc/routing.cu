@@ -428,6 +428,48 @@ __global__ void __launch_bounds__(256) reduce_slots_kernel(const float* __restri
   }
 }
 
+// Owner side of the per-pair return: slot j < k of row t holds the unweighted output
+// row of t's j-th routed expert (sent by the rank that owns that expert), slots
+// k .. k + n_extra - 1 the shared expert's shares; the sum takes the same order as
+// the one-GPU combine (fused multiply-adds over j ascending, then the shared rows),
+// so on one rank it equals the plain forward bit for bit.
+__global__ void __launch_bounds__(256) reduce_pairs_kernel(const float* __restrict__ slab, int k,
+                                                           int n_extra, int rows, int H,
+                                                           const float* __restrict__ w,
+                                                           const uint8_t* __restrict__ valid,
+                                                           __nv_bfloat16* __restrict__ out) {
+  const int nv = H / 8;
+  const size_t per_slot = (size_t)rows * H;
+  for (int t = blockIdx.x; t < rows; t += gridDim.x) {
+    const bool ok = valid == nullptr || valid[t];
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * H);
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (ok) {
+        for (int j = 0; j < k + n_extra; ++j) {
+          const float4* src =
+              reinterpret_cast<const float4*>(slab + j * per_slot + (size_t)t * H) + 2 * v;
+          const float4 a = src[0], b = src[1];
+          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          if (j < k) {
+            const float wj = w[(size_t)t * k + j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += f[i];
+          }
+        }
+      }
+      uint4 o;
+      __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      dst[v] = o;
+    }
+  }
+}
+
 // FP8 path, activation quantisation: a warp takes up to four 1x128 groups of one
 // valid token (their loads issued together), computes for each s = amax / 448 (1 if
 // amax = 0) and the e4m3 codes of x / s (fp32 division, round to nearest even,
@@ -575,6 +617,14 @@ cudaError_t launch_reduce_slots(const float* slots, int n_slots, int rows, int H
   int grid = rows < 148 * 16 ? rows : 148 * 16;
   if (grid < 1) grid = 1;
   reduce_slots_kernel<<<grid, 256, 0, st>>>(slots, n_slots, rows, H, valid, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_pairs(const float* slab, int k, int n_extra, int rows, int H,
+                                const float* w, const uint8_t* valid, __nv_bfloat16* out,
+                                cudaStream_t st) {
+  const int grid = rows < 4096 ? rows : 4096;
+  reduce_pairs_kernel<<<grid, 256, 0, st>>>(slab, k, n_extra, rows, H, w, valid, out);
   return cudaGetLastError();
 }
 

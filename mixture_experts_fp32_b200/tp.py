@@ -33,6 +33,15 @@ return for the combine's all-to-all, so no kernel waits on another (the down GEM
 per-expert completion signals of an all-to-all combine are not needed: the return rides
 in the layer's last kernel).
 
+Per-pair return ("pairs", expert-parallel layout; the Single Batch Overlap of the
+[SGLang] MoE 모델을 위한 Single Batch Overlap 기법 page): the shared expert is computed
+whole by every rank on its own rows, while its all_gather (the dispatch) is in flight;
+the routed experts' down GEMM raises a completion counter per expert, and sender CTAs
+of the same launch copy each finished expert's output rows, unweighted, into slot j of
+the owning rank's slab as soon as that expert is done (`moe_forward_scatter_pairs`);
+the owner then sums its k slots with its routing weights in the one-GPU order, plus
+the shared row (`moe_reduce_pairs`).
+
 Row ownership: gathered row t belongs to rank t // rows, local row t % rows.
 """
 from __future__ import annotations
@@ -156,6 +165,28 @@ class LibraryKernels:
         moe.moe_reduce_partials(slab, n_slots, rows, H, valid, out)
 
 
+class SharedOwnRows:
+    """The shared expert of the per-pair layout, whole, on a rank's own rows: a
+    one-expert layer whose router always picks that expert with weight exactly 1
+    (zero router weights), returned unrounded into the rank's own slab."""
+
+    def __init__(self, full: dict, *, H: int, Is: int, rows: int, fp8: bool, device):
+        self.plan = moe.Plan(max_tokens=rows, hidden=H, num_experts=1, top_k_max=1, inter=Is,
+                             wtype=moe.MOE_W_FP8_E4M3_B128 if fp8 else moe.MOE_W_BF16,
+                             device=device)
+        self.router_w = torch.zeros(1, H, dtype=torch.float32, device=device)
+        self.w_gate_up = full["ws_gate_up"][None].contiguous()
+        self.w_down = full["ws_down"][None].contiguous()
+        self.s_gate_up = full["ss_gate_up"][None].contiguous() if fp8 else None
+        self.s_down = full["ss_down"][None].contiguous() if fp8 else None
+        self.weights = self.plan.weights(self.router_w, None, self.w_gate_up, self.w_down,
+                                         self.s_gate_up, self.s_down)
+
+    def forward(self, x_local, valid_local, dst_ptr: int, rows: int, stream=None):
+        self.plan.forward_scatter(self.weights, x_local, valid_local, 1, [dst_ptr], rows, 0,
+                                  stream=stream)
+
+
 class TPMoE:
     """One rank of the tensor-parallel layer (layout "tp") or of the expert-parallel one
     (layout "ep").  `full` holds the whole layer's weights on this rank's device (the
@@ -170,7 +201,8 @@ class TPMoE:
 
     def __init__(self, full: dict, *, E: int, H: int, I: int, S: int, Is: int, k_max: int,
                  rows: int, fp8: bool = False, fused: bool = True, group=None,
-                 barrier_timeout_ms: int = 10000, layout: str = "tp", kernels=LibraryKernels):
+                 barrier_timeout_ms: int = 10000, layout: str = "tp", kernels=LibraryKernels,
+                 pairs: bool = False, send_ctas: int = 16):
         import torch.distributed as dist
         self.group = group if group is not None else dist.group.WORLD
         self.n = dist.get_world_size(group)
@@ -179,6 +211,11 @@ class TPMoE:
             raise ValueError("at most 8 tensor-parallel ranks")
         self.H, self.rows, self.fused = H, rows, fused
         self.timeout_ms = barrier_timeout_ms
+        self.pairs = pairs
+        if pairs:
+            self._init_pairs(full, E=E, H=H, I=I, S=S, Is=Is, k_max=k_max, rows=rows, fp8=fp8,
+                             send_ctas=send_ctas)
+            return
         if layout == "tp":
             self.shard = shard_weights(full, self.n, self.rank, I=I, Is=Is, fp8=fp8)
             self.experts, inter = (0, E), I // self.n
@@ -209,6 +246,65 @@ class TPMoE:
             self.partial = torch.empty(T, H, dtype=torch.float32, device=dev)
             self.recv = torch.empty(rows, H, dtype=torch.float32, device=dev)
 
+    def _init_pairs(self, full, *, E, H, I, S, Is, k_max, rows, fp8, send_ctas):
+        """Expert-parallel layout with the per-pair return: this rank's routed experts
+        whole (no shared expert in that plan), the shared expert whole on its own rows,
+        and a slab of k_max + 1 slots per owner (two, used on alternate steps)."""
+        import torch.distributed._symmetric_memory as symm
+        dev = full["w_gate_up"].device
+        self.experts = expert_range(E, self.n, self.rank)
+        e0, e1 = self.experts
+        self.shard = {"router_w": full["router_w"], "router_b": full.get("router_b"),
+                      "w_gate_up": full["w_gate_up"][e0:e1].contiguous(),
+                      "w_down": full["w_down"][e0:e1].contiguous()}
+        if fp8:
+            self.shard["s_gate_up"] = full["s_gate_up"][e0:e1].contiguous()
+            self.shard["s_down"] = full["s_down"][e0:e1].contiguous()
+        T = self.n * rows
+        self.kernels = LibraryKernels(self.shard, E=E, H=H, inter=I, S=0, shared_inter=0,
+                                      k_max=k_max, T=T, fp8=fp8, device=dev)
+        self.shared = (SharedOwnRows(full, H=H, Is=Is, rows=rows, fp8=fp8, device=dev)
+                       if S else None)
+        self.k_max, self.send_ctas = k_max, send_ctas
+        self.x_all = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.valid_all = torch.empty(T, dtype=torch.uint8, device=dev)
+        self.w_all = torch.empty(T, k_max, dtype=torch.float32, device=dev)
+        self.step = 0
+        self.slab = symm.empty(2, k_max + 1, rows, H, dtype=torch.float32, device=dev)
+        self.handle = symm.rendezvous(self.slab, self.group)
+        base = [int(p) for p in self.handle.buffer_ptrs]
+        per = (k_max + 1) * rows * H * 4
+        self.dst = [[b + par * per for b in base] for par in range(2)]
+        self.comm = torch.cuda.Stream(device=dev)
+
+    def _forward_pairs(self, x_local, valid_local, k: int, out_local):
+        import torch.distributed as dist
+        if k != self.k_max:
+            raise ValueError("the per-pair slabs and weights are laid out for k = k_max")
+        par = self.step & 1
+        main = torch.cuda.current_stream()
+        # the dispatch (all_gather) on the communication stream, while the shared
+        # expert runs on this rank's own rows
+        self.comm.wait_stream(main)
+        with torch.cuda.stream(self.comm):
+            dist.all_gather_into_tensor(self.x_all, x_local, group=self.group)
+            dist.all_gather_into_tensor(self.valid_all, valid_local, group=self.group)
+        n_extra = 0
+        if self.shared is not None:
+            own = self.dst[par][self.rank] + self.k_max * self.rows * self.H * 4
+            self.shared.forward(x_local, valid_local, own, self.rows)
+            n_extra = 1
+        main.wait_stream(self.comm)
+        dbg = moe.make_debug(topk_w=self.w_all)
+        self.kernels.plan.forward_scatter_pairs(self.kernels.weights, self.x_all, self.valid_all,
+                                                k, self.dst[par], self.rows, k, *self.experts,
+                                                self.send_ctas, dbg=dbg)
+        self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
+        lo = self.rank * self.rows
+        moe.moe_reduce_pairs(self.slab[par], k, n_extra, self.rows, self.H,
+                             self.w_all[lo:lo + self.rows], valid_local, out_local)
+        self.step += 1
+
     @property
     def plan(self):
         return self.kernels.plan
@@ -237,6 +333,9 @@ class TPMoE:
 
     def forward(self, x_local, valid_local, k: int, out_local):
         """x_local bf16 [rows, H], valid_local uint8 [rows], out_local bf16 [rows, H]."""
+        if self.pairs:
+            self._forward_pairs(x_local, valid_local, k, out_local)
+            return
         self._gather(x_local, valid_local)
         self._compute_and_return(k, valid_local, out_local)
 
@@ -266,6 +365,52 @@ class TPMoETwoBatch:
             main.wait_event(e)
             half._compute_and_return(k, valid_local[lo:hi], out_local[lo:hi])
         main.wait_stream(self.comm)
+
+
+def pairs_forward_reference(full: dict, x_rows: List[torch.Tensor],
+                            valid_rows: List[torch.Tensor], k: int, *, E, H, I, S, Is, fp8,
+                            n_shards: int, send_ctas: int = 16):
+    """One-GPU emulation of n expert-parallel ranks with the per-pair return (no
+    process group): each rank's shared expert on its own rows into its own slab,
+    each rank's routed experts sent into every owner's slab, then each owner's
+    reduction.  Returns the owners' outputs."""
+    dev = full["w_gate_up"].device
+    rows = x_rows[0].shape[0]
+    x_all = torch.cat(x_rows)
+    v_all = torch.cat(valid_rows)
+    T = n_shards * rows
+    slabs = [torch.full((k + 1, rows, H), float("nan"), dtype=torch.float32, device=dev)
+             for _ in range(n_shards)]
+    w_all = torch.empty(T, k, dtype=torch.float32, device=dev)
+    keep, kerns = [], []
+    for r in range(n_shards):
+        if S:
+            sh = SharedOwnRows(full, H=H, Is=Is, rows=rows, fp8=fp8, device=dev)
+            sh.forward(x_rows[r], valid_rows[r], slabs[r][k].data_ptr(), rows)
+            keep.append(sh)
+        e0, e1 = expert_range(E, n_shards, r)
+        shard = {"router_w": full["router_w"], "router_b": full.get("router_b"),
+                 "w_gate_up": full["w_gate_up"][e0:e1].contiguous(),
+                 "w_down": full["w_down"][e0:e1].contiguous()}
+        if fp8:
+            shard["s_gate_up"] = full["s_gate_up"][e0:e1].contiguous()
+            shard["s_down"] = full["s_down"][e0:e1].contiguous()
+        kern = LibraryKernels(shard, E=E, H=H, inter=I, S=0, shared_inter=0, k_max=k, T=T,
+                              fp8=fp8, device=dev)
+        kern.plan.forward_scatter_pairs(kern.weights, x_all, v_all, k, slabs, rows, k, e0, e1,
+                                        send_ctas, dbg=moe.make_debug(topk_w=w_all))
+        kerns.append(kern)
+        keep.append(shard)
+    outs = []
+    for r in range(n_shards):
+        o = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+        moe.moe_reduce_pairs(slabs[r], k, 1 if S else 0, rows, H, w_all[r * rows:(r + 1) * rows],
+                             valid_rows[r], o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    statuses = [kern.plan.device_status() for kern in kerns]
+    statuses += [sh.plan.device_status() for sh in keep if isinstance(sh, SharedOwnRows)]
+    return outs, statuses
 
 
 def tp_forward_reference(full: dict, x_rows: List[torch.Tensor], valid_rows: List[torch.Tensor],

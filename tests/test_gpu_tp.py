@@ -125,3 +125,101 @@ def test_one_rank_two_micro_batches(one_rank_group):
         sub["workload"] = w.with_(T=hi - lo)
         ref = run_forward(plan_for(sub["workload"]), sub, w.k)["out"]
         assert torch.equal(out[lo:hi].cpu().view(torch.int16), ref.view(torch.int16))
+
+
+# ----------------------------------------------------- per-pair return (signalled sends)
+
+PAIR_CASES = [
+    (Workload("pairs1_bf16_padded", T=64, H=512, E=16, k=3, I=256, S=1, Is=256,
+              router_sigma=0.2, mask="dp_padded", dp_rows=(40,)), 1),
+    (Workload("pairs2_bf16_padded", T=4 * 48, H=512, E=16, k=3, I=256, S=1, Is=256,
+              router_sigma=0.2, mask="dp_padded", dp_rows=(48, 5, 0, 17)), 2),
+    (Workload("pairs4_bf16_zipf", T=4 * 64, H=512, E=16, k=4, I=256, S=1, Is=512,
+              router_sigma=0.2, bias="zipf"), 4),
+    (Workload("pairs2_fp8", T=2 * 64, H=512, E=8, k=2, I=256, S=1, Is=256, wtype="fp8",
+              router_sigma=0.2, w_sigma=0.05), 2),
+    (Workload("pairs4_fp8_no_shared", T=4 * 32, H=512, E=8, k=3, I=256, S=0, Is=0,
+              wtype="fp8", router_sigma=0.2, w_sigma=0.05), 4),
+    (Workload("pairs2_bf16_many_rows", T=2 * 400, H=256, E=4, k=2, I=256, S=1, Is=128,
+              router_sigma=0.2), 2),                      # several row tiles per expert
+]
+
+
+@pytest.mark.parametrize("w,n", PAIR_CASES, ids=lambda c: c.name if hasattr(c, "name") else str(c))
+def test_emulated_pairs_return_matches_the_layer(w, n):
+    """Each emulated expert-parallel rank computes the shared expert whole on its own
+    rows and sends its routed experts' rows, one slot per pair, into the owners' slabs
+    from the sender CTAs of its down GEMM; each owner's ordered sum is the one-GPU
+    combine, so the owners' outputs equal the unsharded forward bit for bit (and the
+    oracle within the layer's tolerance)."""
+    inp = synth.make_inputs(w)
+    d = to_device(inp)
+    rows = w.T // n
+    full_res = run_forward(plan_for(w), d, w.k)
+    xs = [d["x"][r * rows:(r + 1) * rows] for r in range(n)]
+    vs = [d["valid"][r * rows:(r + 1) * rows] for r in range(n)]
+    for send_ctas in (1, 16):
+        outs, statuses = tp.pairs_forward_reference(d, xs, vs, w.k, E=w.E, H=w.H, I=w.I, S=w.S,
+                                                    Is=w.Is, fp8=w.wtype == "fp8", n_shards=n,
+                                                    send_ctas=send_ctas)
+        assert all(s == 0 for s in statuses), statuses
+        got = torch.cat(outs).cpu()
+        res = dict(full_res)
+        res["out"] = got
+        check_against_oracle(inp, res, w.k)
+        assert torch.equal(got.view(torch.int16), full_res["out"].view(torch.int16))
+
+
+def test_pairs_sender_wait_limit_sets_the_status_bit():
+    """With a zero wait limit every wait not already satisfied gives up at once: the
+    senders set MOE_DEV_WAIT_TIMEOUT_SEND and stop, the launch still ends, and the
+    same plan then runs correctly with the normal limit."""
+    w = Workload("pairs_timeout", T=2 * 64, H=512, E=8, k=2, I=256, S=0, Is=0,
+                 router_sigma=0.2)
+    inp = synth.make_inputs(w)
+    d = to_device(inp)
+    rows = w.T // 2
+    shard = {"router_w": d["router_w"], "router_b": d.get("router_b"),
+             "w_gate_up": d["w_gate_up"], "w_down": d["w_down"]}
+    kern = tp.LibraryKernels(shard, E=w.E, H=w.H, inter=w.I, S=0, shared_inter=0, k_max=w.k,
+                             T=w.T, fp8=False, device=d["x"].device)
+    slabs = [torch.zeros(w.k + 1, rows, w.H, dtype=torch.float32, device="cuda")
+             for _ in range(2)]
+    kern.plan.set_wait_limit(0)
+    kern.plan.forward_scatter_pairs(kern.weights, d["x"], d["valid"], w.k, slabs, rows, w.k,
+                                    0, w.E, 8)
+    torch.cuda.synchronize()
+    bits = kern.plan.device_status()
+    assert bits & moe.MOE_DEV_WAIT_TIMEOUT_SEND, hex(bits)
+    kern.plan.set_wait_limit(2_000_000_000)
+    wts = torch.empty(w.T, w.k, dtype=torch.float32, device="cuda")
+    kern.plan.forward_scatter_pairs(kern.weights, d["x"], d["valid"], w.k, slabs, rows, w.k,
+                                    0, w.E, 8, dbg=moe.make_debug(topk_w=wts))
+    torch.cuda.synchronize()
+    assert kern.plan.device_status() == 0
+    ref = run_forward(plan_for(w), d, w.k)["out"]
+    for r in range(2):
+        o = torch.empty(rows, w.H, dtype=torch.bfloat16, device="cuda")
+        moe.moe_reduce_pairs(slabs[r], w.k, 0, rows, w.H, wts[r * rows:(r + 1) * rows],
+                             d["valid"][r * rows:(r + 1) * rows], o)
+        torch.cuda.synchronize()
+        assert torch.equal(o.cpu().view(torch.int16), ref[r * rows:(r + 1) * rows].view(torch.int16))
+
+
+def test_one_rank_pairs_layer_equals_the_layer(one_rank_group):
+    """TPMoE with the per-pair return on a one-rank group: the all_gather on the
+    communication stream while the shared expert runs on the rank's own rows, the
+    signalled sends into the symmetric-memory slab, the barrier and the owner's sum
+    give the unsharded forward's output bit for bit, step after step."""
+    w = Workload("pairs1_layer", T=64, H=512, E=16, k=3, I=512, S=1, Is=256, router_sigma=0.2,
+                 mask="dp_padded", dp_rows=(40,))
+    d = to_device(synth.make_inputs(w))
+    ref = run_forward(plan_for(w), d, w.k)["out"]
+    layer = tp.TPMoE(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is, k_max=w.k, rows=w.T,
+                     fp8=False, layout="ep", pairs=True, send_ctas=8)
+    for _ in range(3):
+        out = torch.full((w.T, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        layer.forward(d["x"], d["valid"], w.k, out)
+        torch.cuda.synchronize()
+        assert layer.plan.device_status() == 0
+        assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
