@@ -325,13 +325,13 @@ __device__ __forceinline__ float elem8(const Vec8<__nv_bfloat16>& v, int i) {
 
 // MAXKS bounds k + S at compile time, so that the variant for up to four rows a token
 // (decode: top-3 with a shared expert) keeps only four row vectors in registers and
-// runs at twice the occupancy of the general one.
+// runs at twice the occupancy of the general one.  With bf16 expert outputs (FP8
+// weights) the registers are capped for three resident blocks an SM.
 template <typename YT, bool F32OUT, int MAXKS>
-__global__ void __launch_bounds__(256) combine_kernel(const YT* __restrict__ y, int H,
-                                                      const int* __restrict__ inv,
-                                                      const float* __restrict__ w,
-                                                      const uint8_t* __restrict__ valid, int T,
-                                                      int k, int S, const CombineOut co) {
+__global__ void __launch_bounds__(256, sizeof(YT) == 2 ? 3 : 1)
+    combine_kernel(const YT* __restrict__ y, int H, const int* __restrict__ inv,
+                   const float* __restrict__ w, const uint8_t* __restrict__ valid, int T, int k,
+                   int S, const CombineOut co) {
   __shared__ int rows[kMaxTopK + 1];
   __shared__ float wts[kMaxTopK];
   const int ks = k + S;
