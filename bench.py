@@ -40,7 +40,7 @@ L2_FLUSH_BYTES = 512 << 20
 # capture of that kernel on the Step3 decode shape (8 experts, 1 GPU); it applies
 # only to the kernel source it was measured on (sha256 prefix), and "traffic" is
 # null otherwise.
-GEMM_TRAFFIC = {"sha256_prefix": "0ed45de09043589f", "gate_up_ratio": 0.998}
+GEMM_TRAFFIC = {"sha256_prefix": "5a12df72098ca22e", "gate_up_ratio": 1.000}
 
 
 def gemm_source_hash() -> str:
@@ -758,9 +758,12 @@ def cpu_baseline(w, inp, gpu, target_s: float):
     return out
 
 
-def tp_reference_rows(d, w, rank: int, rows: int, dev):
-    """Rows [rank * rows, (rank + 1) * rows) of one GPU's plain forward of the whole
-    gathered batch, computed before the layer is sharded."""
+def tp_reference_rows(d, w, rank: int, n_ranks: int, rows: int, ranges, dev):
+    """This rank's rows [rank * rows, (rank + 1) * rows) as one GPU's plain forward
+    computes them, before the layer is sharded: one forward per micro-batch, over the
+    rows that micro-batch gathers from every rank (`ranges`: each micro-batch's
+    [lo, hi) within a rank's rows), so that on one rank the layer must match it bit
+    for bit (the router's split of its sums depends on the number of rows)."""
     import torch
 
     import mixture_experts_fp32_b200 as moe
@@ -770,13 +773,17 @@ def tp_reference_rows(d, w, rank: int, rows: int, dev):
     wts = plan.weights(d["router_w"], d["router_b"], d["w_gate_up"], d["w_down"],
                        d.get("s_gate_up"), d.get("s_down"), d.get("ws_gate_up"),
                        d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
-    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
-    plan.forward(wts, d["x"], d["valid"], w.k, out)
+    mine = torch.empty(rows, w.H, dtype=torch.bfloat16, device=dev)
+    for lo, hi in ranges:
+        idx = torch.cat([torch.arange(r * rows + lo, r * rows + hi, device=dev)
+                         for r in range(n_ranks)])
+        out = torch.empty(len(idx), w.H, dtype=torch.bfloat16, device=dev)
+        plan.forward(wts, d["x"][idx].contiguous(), d["valid"][idx].contiguous(), w.k, out)
+        mine[lo:hi] = out[rank * (hi - lo):(rank + 1) * (hi - lo)]
     torch.cuda.synchronize()
     if plan.device_status() != 0:
         raise RuntimeError("device status set in the one-GPU reference forward")
-    mine = out[rank * rows:(rank + 1) * rows].clone()
-    del plan, wts, out
+    del plan, wts
     torch.cuda.empty_cache()
     return mine
 
@@ -842,14 +849,17 @@ def run_tp(args):
         d = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
         del inp
         valid_tokens = int(d["valid"].sum().item())
-        # the reference for this rank's rows: one GPU's plain forward of the gathered batch
-        ref_rows = tp_reference_rows(d, w, rank, rows, dev)
+        two = args.tp_microbatches == 2 and rows >= 2
+        # the reference for this rank's rows: one GPU's plain forward of what each
+        # micro-batch gathers
+        ref_rows = tp_reference_rows(d, w, rank, ws_n, rows,
+                                     tp.split_rows(rows) if two else [(0, rows)], dev)
         pairs = args.tp_return == "pairs"
         kw = dict(E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is if w.S else 0, k_max=w.k,
                   fp8=w.wtype == "fp8", fused=args.tp_return != "nccl",
                   layout="ep" if pairs else args.tp_layout, pairs=pairs,
                   send_ctas=args.send_ctas)
-        if args.tp_microbatches == 2 and rows >= 2:
+        if two:
             layer = tp.TPMoETwoBatch(d, rows=rows, **kw)
         else:
             layer = tp.TPMoE(d, rows=rows, **kw)

@@ -278,32 +278,35 @@ class TPMoE:
         self.comm = torch.cuda.Stream(device=dev)
 
     def _forward_pairs(self, x_local, valid_local, k: int, out_local):
-        import torch.distributed as dist
-        if k != self.k_max:
-            raise ValueError("the per-pair slabs and weights are laid out for k = k_max")
-        par = self.step & 1
         main = torch.cuda.current_stream()
         # the dispatch (all_gather) on the communication stream, while the shared
         # expert runs on this rank's own rows
         self.comm.wait_stream(main)
         with torch.cuda.stream(self.comm):
-            dist.all_gather_into_tensor(self.x_all, x_local, group=self.group)
-            dist.all_gather_into_tensor(self.valid_all, valid_local, group=self.group)
-        n_extra = 0
-        if self.shared is not None:
-            own = self.dst[par][self.rank] + self.k_max * self.rows * self.H * 4
-            self.shared.forward(x_local, valid_local, own, self.rows)
-            n_extra = 1
+            self._gather(x_local, valid_local)
+        self._shared_own(x_local, valid_local)
         main.wait_stream(self.comm)
+        self._compute_and_return(k, valid_local, out_local)
+
+    def _shared_own(self, x_local, valid_local):
+        """Per-pair layout: the shared expert on this rank's own rows, into its own
+        slab's last slot (nothing without a shared expert or in the other layouts)."""
+        if self.pairs and self.shared is not None:
+            own = self.dst[self.step & 1][self.rank] + self.k_max * self.rows * self.H * 4
+            self.shared.forward(x_local, valid_local, own, self.rows)
+
+    def _return_pairs(self, k: int, valid_local, out_local):
+        if k != self.k_max:
+            raise ValueError("the per-pair slabs and weights are laid out for k = k_max")
+        par = self.step & 1
         dbg = moe.make_debug(topk_w=self.w_all)
         self.kernels.plan.forward_scatter_pairs(self.kernels.weights, self.x_all, self.valid_all,
                                                 k, self.dst[par], self.rows, k, *self.experts,
                                                 self.send_ctas, dbg=dbg)
         self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
         lo = self.rank * self.rows
-        moe.moe_reduce_pairs(self.slab[par], k, n_extra, self.rows, self.H,
-                             self.w_all[lo:lo + self.rows], valid_local, out_local)
-        self.step += 1
+        moe.moe_reduce_pairs(self.slab[par], k, 1 if self.shared is not None else 0, self.rows,
+                             self.H, self.w_all[lo:lo + self.rows], valid_local, out_local)
 
     @property
     def plan(self):
@@ -315,8 +318,12 @@ class TPMoE:
         dist.all_gather_into_tensor(self.valid_all, valid_local, group=self.group)
 
     def _compute_and_return(self, k: int, valid_local, out_local):
+        """The layer over the gathered rows and the return of the partial sums (after
+        `_gather`, and for the per-pair layout after `_shared_own`)."""
         import torch.distributed as dist
-        if self.fused:
+        if self.pairs:
+            self._return_pairs(k, valid_local, out_local)
+        elif self.fused:
             par = self.step & 1
             self.kernels.forward_scatter_experts(self.x_all, self.valid_all, k, self.dst[par],
                                                  self.rows, self.rank, *self.experts)
@@ -362,6 +369,7 @@ class TPMoETwoBatch:
                 e.record(self.comm)
                 ev.append(e)
         for e, (lo, hi), half in zip(ev, self.ranges, self.halves):
+            half._shared_own(x_local[lo:hi], valid_local[lo:hi])
             main.wait_event(e)
             half._compute_and_return(k, valid_local[lo:hi], out_local[lo:hi])
         main.wait_stream(self.comm)

@@ -36,8 +36,8 @@ def sample_rows(valid: np.ndarray, n_random: int = 6, seed: int = 0) -> np.ndarr
 
 
 def tile_rows(offsets: np.ndarray, E: int, S: int, valid: np.ndarray, heavy: int = 3,
-              small: int = 4) -> np.ndarray:
-    """Permuted row indices: the first row of every 128-row tile of the `heavy`
+              small: int = 4, stride: int = 128) -> np.ndarray:
+    """Permuted row indices: the first row of every `stride`-row tile of the `heavy`
     largest routed groups and of the shared group (rows past offsets[E]), the last
     row of each such group, and the first row of `small` groups of 1..64 rows."""
     counts = np.diff(offsets)
@@ -48,7 +48,7 @@ def tile_rows(offsets: np.ndarray, E: int, S: int, valid: np.ndarray, heavy: int
         groups.append((offsets[-1], offsets[-1] + nv))            # the shared group
     rows = []
     for b, e in groups:
-        rows += list(range(b, e, 128)) + [e - 1]
+        rows += list(range(b, e, stride)) + [e - 1]
     tiny = [e for e in range(E) if 0 < counts[e] <= 64][:small]
     rows += [offsets[e] for e in tiny]
     return np.unique(np.asarray(rows, dtype=np.int64))
@@ -163,7 +163,8 @@ def test_full_size_workload(name):
     res = run_forward(plan, d, w.k)
     valid = inp["valid"].numpy()
     offsets = res["offsets"].numpy()
-    prow = tile_rows(offsets, w.E, w.S, valid)
+    # tiles of 128 rows (FP8 GEMMs, bf16 gate/up); the bf16 down GEMM's are 96
+    prow = tile_rows(offsets, w.E, w.S, valid, stride=128 if w.wtype == "fp8" else 96)
     perm = res["perm"].numpy()
     # the tokens behind those permuted rows (shared rows: the valid tokens in order)
     vi = np.nonzero(valid)[0]

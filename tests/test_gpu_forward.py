@@ -28,6 +28,8 @@ CASES = [
     W("e256_k8_bias", T=200, H=256, E=256, k=8, I=128, S=1, Is=128, bias="normal"),
     W("two_row_tiles", T=300, H=256, E=2, k=1, I=128),            # ~150 rows per expert
     W("skewed", T=300, H=256, E=4, k=2, I=256, bias="zipf", zipf_s=3.0),   # > 256 rows on one
+    # a decode-sized batch whose Zipf load puts 46 and 62 rows on two of 16 experts
+    W("decode_skewed", T=64, H=256, E=16, k=2, I=128, S=1, Is=128, bias="zipf", zipf_s=2.0),
     W("k_equals_e", T=9, H=256, E=4, k=4, I=128),
     W("padded", T=64, H=256, E=8, k=2, I=128, S=1, Is=128, mask="dp_padded",
       dp_rows=(3, 16, 0, 5)),

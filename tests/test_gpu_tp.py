@@ -110,21 +110,31 @@ def test_one_rank_tp_equals_the_layer(one_rank_group, fused, layout):
         assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
 
 
-def test_one_rank_two_micro_batches(one_rank_group):
+@pytest.mark.parametrize("kw", [dict(fused=True), dict(fused=False),
+                                dict(fused=True, layout="ep"),
+                                dict(fused=True, layout="ep", pairs=True, send_ctas=8)],
+                         ids=["tp-fused", "tp-nccl", "ep-fused", "ep-pairs"])
+def test_one_rank_two_micro_batches(one_rank_group, kw):
+    """Two micro-batches on one rank, in every return form (the per-pair one with its
+    shared expert on the rank's own rows of each micro-batch): each micro-batch's
+    rows equal the plain forward of that micro-batch, bit for bit, step after step."""
     w = Workload("tp1_tbo", T=96, H=512, E=16, k=3, I=512, S=1, Is=256, router_sigma=0.2,
                  mask="dp_padded", dp_rows=(70,))
     d = to_device(synth.make_inputs(w))
-    layer = tp.TPMoETwoBatch(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is, k_max=w.k, rows=w.T,
-                             fp8=False, fused=True)
-    out = torch.full((w.T, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
-    layer.forward(d["x"], d["valid"], w.k, out)
-    torch.cuda.synchronize()
-    for (lo, hi) in layer.ranges:                        # each micro-batch is its own layer call
+    refs = []
+    for (lo, hi) in tp.split_rows(w.T):                  # each micro-batch is its own layer call
         sub = dict(d)
         sub["x"], sub["valid"] = d["x"][lo:hi], d["valid"][lo:hi]
-        sub["workload"] = w.with_(T=hi - lo)
-        ref = run_forward(plan_for(sub["workload"]), sub, w.k)["out"]
-        assert torch.equal(out[lo:hi].cpu().view(torch.int16), ref.view(torch.int16))
+        refs.append(run_forward(plan_for(w.with_(T=hi - lo)), sub, w.k)["out"])
+    layer = tp.TPMoETwoBatch(d, E=w.E, H=w.H, I=w.I, S=w.S, Is=w.Is, k_max=w.k, rows=w.T,
+                             fp8=False, **kw)
+    for _ in range(3):                                   # alternate slabs across steps
+        out = torch.full((w.T, w.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        layer.forward(d["x"], d["valid"], w.k, out)
+        torch.cuda.synchronize()
+        assert all(h.plan.device_status() == 0 for h in layer.halves)
+        for (lo, hi), ref in zip(layer.ranges, refs):
+            assert torch.equal(out[lo:hi].cpu().view(torch.int16), ref.view(torch.int16))
 
 
 # ----------------------------------------------------- per-pair return (signalled sends)
