@@ -142,6 +142,23 @@ def launches_per_step(w) -> int:
     return 2 + route + 1 + 2 + 1
 
 
+def tp_launches_per_step(w, n_ranks: int, rows: int, n_mb: int, ret: str) -> int:
+    """This library's kernels one step of the tensor- / expert-parallel layer launches
+    (NCCL's and the symmetric-memory barrier's not counted): per micro-batch the
+    layer over the gathered rows and the owner's reduction; with the per-pair return
+    the combine is replaced by the sends inside the down GEMM, and the shared expert
+    runs on the rank's own rows as a one-expert layer (router, top-k, one route
+    kernel, gather, two GEMMs, combine)."""
+    total = 0
+    for lo, hi in ([(0, rows // 2), (rows // 2, rows)] if n_mb == 2 else [(0, rows)]):
+        layer = launches_per_step(w.with_(T=n_ranks * (hi - lo)))
+        if ret == "pairs":
+            total += (layer - 1) + 1 + (7 if w.S else 0)
+        else:
+            total += layer + 1
+    return total
+
+
 def step_spread(ms) -> dict:
     """Median and 10th / 90th percentiles (linear interpolation) of per-step times."""
     import numpy as np
@@ -849,7 +866,8 @@ def run_tp(args):
         d = {key: (v.to(dev) if isinstance(v, torch.Tensor) else v) for key, v in inp.items()}
         del inp
         valid_tokens = int(d["valid"].sum().item())
-        two = args.tp_microbatches == 2 and rows >= 2
+        n_mb = args.tp_microbatches or (2 if w.wtype == "fp8" else 1)
+        two = n_mb == 2 and rows >= 2
         # the reference for this rank's rows: one GPU's plain forward of what each
         # micro-batch gathers
         ref_rows = tp_reference_rows(d, w, rank, ws_n, rows,
@@ -888,6 +906,28 @@ def run_tp(args):
         if flag.item() != 0.0:
             raise RuntimeError(f"tensor-parallel rows differ from the one-GPU forward: {check}")
         K = args.steps
+        # end to end through the layer's Python API: each step uploads this rank's rows
+        # and mask from pinned host memory and downloads its output to pinned host memory
+        x_host = x_loc.cpu().pin_memory()
+        v_host = v_loc.cpu().pin_memory()
+        o_host = torch.empty(rows, w.H, dtype=torch.bfloat16).pin_memory()
+        x_dev, v_dev = torch.empty_like(x_loc), torch.empty_like(v_loc)
+        e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(K)]
+        dist.barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in e2e_ev:
+            e0.record()
+            x_dev.copy_(x_host, non_blocking=True)
+            v_dev.copy_(v_host, non_blocking=True)
+            layer.forward(x_dev, v_dev, w.k, out)
+            o_host.copy_(out, non_blocking=True)
+            e1.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = reduce_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / K, "max", ws_n,
+                                   dev)
+        e2e_ok = bool(torch.equal(o_host.view(torch.int16), out.cpu().view(torch.int16)))
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
         clocks = ClockSampler(dev.index)
@@ -921,7 +961,18 @@ def run_tp(args):
                            "send_ctas": args.send_ctas if pairs else None,
                            "micro_batches": 2 if hasattr(layer, "halves") else 1,
                            "l2": f"{L2_FLUSH_BYTES >> 20} MB written between timed steps"},
-                "check": check, "gpu_launches": None, "clocks": clk}))
+                "check": check,
+                "e2e": {"value": valid_tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                        "ms_per_step": e2e_ms,
+                        "h2d_bytes_per_step": ws_n * (x_host.numel() * 2 + v_host.numel()),
+                        "d2h_bytes_per_step": ws_n * o_host.numel() * 2,
+                        "output_matches_device": e2e_ok,
+                        "how": "TP layer's forward with each rank's rows and mask uploaded "
+                               "from pinned host memory and its output downloaded every "
+                               "step (CUDA events, max over ranks, L2 not flushed)"},
+                "gpu_launches": K * tp_launches_per_step(w, ws_n, rows, 2 if two else 1,
+                                                         args.tp_return),
+                "clocks": clk}))
     finally:
         del layer
         torch.cuda.synchronize()
@@ -1020,7 +1071,10 @@ def main(argv=None):
     ap.add_argument("--tp-layout", default="tp", choices=["tp", "ep"],
                     help="with --tp: split every expert's intermediate dimension (tp) or "
                          "the experts (ep) over the ranks")
-    ap.add_argument("--tp-microbatches", type=int, default=2, choices=[1, 2])
+    ap.add_argument("--tp-microbatches", type=int, default=0, choices=[0, 1, 2],
+                    help="with --tp: micro-batches per step; 0 = one for the HBM-bound bf16 "
+                         "decode batches (each micro-batch streams the rank's weights once), "
+                         "two for the FP8 prefill")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the number of routed experts (profiling on a smaller case)")
     args = ap.parse_args(argv)

@@ -54,6 +54,18 @@ def test_launch_count_per_step():
     assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 9
 
 
+def test_tp_launch_count_per_step():
+    w = synth.WORKLOADS["step3_decode"]
+    # one micro-batch: the layer over 8 x 32 gathered rows (7 kernels) + the owner's sum
+    assert bench.tp_launches_per_step(w, 8, 32, 1, "fused") == 8
+    # two micro-batches of 16 rows a rank
+    assert bench.tp_launches_per_step(w, 8, 32, 2, "nccl") == 16
+    # per-pair return: no combine, the pair sum, the shared expert as a one-expert layer
+    assert bench.tp_launches_per_step(w, 8, 32, 1, "pairs") == 6 + 1 + 7
+    # the FP8 prefill gathers 8192 rows: three route kernels and the quantisation
+    assert bench.tp_launches_per_step(synth.WORKLOADS["fp8_prefill"], 8, 1024, 1, "fused") == 10
+
+
 def test_step_spread():
     s = bench.step_spread([float(v) for v in range(1, 12)])     # 1..11 ms
     assert s == {"p10": 2.0, "p50": 6.0, "p90": 10.0}
