@@ -391,7 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                : p.sw_shared;
       // weight scale rows: gated -> gate block and up block of f0; down -> block of this half
       const int up = routed ? p.up_routed : p.up_shared;
-      e.swa = sw + (size_t)((ti.f0 + (GATED ? 0 : hh * 128)) / 128) * ti.k_blocks;
+      // (down: a half past a partial last tile reads its tile's last block, in bounds)
+      e.swa = sw + (size_t)((GATED ? ti.f0 : min(ti.f0 + hh * 128, ti.f0 + ti.nfeat - 1)) / 128) *
+                       ti.k_blocks;
       e.swb = sw + (size_t)((up + ti.f0) / 128) * ti.k_blocks;
       // rows past the group read the tile's first row instead (in bounds, unused)
       e.sa_row = p.sa + (size_t)(r < e.rows ? e.row0 + r : ti.row0) * p.sa_ld;
