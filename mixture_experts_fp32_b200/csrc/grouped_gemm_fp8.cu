@@ -37,7 +37,10 @@
 //          quantised per 1x128 group (the tile's 128 features are one group)
 //          into e4m3 codes and an fp32 scale.
 //   down:  a tile owns up to 256 output features (two weight scale blocks); y
-//          is written in bf16.
+//          is written in bf16, each warp's rows passing through shared memory in
+//          rounds of 8 so that every store covers two whole 256-byte row segments
+//          (one row per thread would make every store touch 32 rows: 8-12 % of the
+//          down GEMM's time on the 8192-token prefill).
 //
 // Signalled sends (down GEMM of an expert-parallel rank): a cooperative launch
 // whose first n_gemm CTAs run the tiles, every epilogue warp counting each stored
@@ -80,7 +83,14 @@ constexpr int STAGES = 4;
 constexpr int DATA_BYTES = STAGES * (A_BYTES + B_BYTES);
 constexpr int RED_BYTES = 2 * BMT * 2 * 4;    // h amax halves [tile parity][row][half]
 constexpr int kGroupSlots = kMaxExperts + 4;   // >= groups + 1
-constexpr int SMEM_BYTES = DATA_BYTES + RED_BYTES + 1024 + 256 + 2 * 4 * kGroupSlots;
+// down: y rows staged per warp, 8 rows x 256 bytes, so that stores cover whole rows
+// (the gated kernel has no staging, which leaves it more L1)
+constexpr int STG_BYTES = kEpiWarps * 8 * 256;
+template <bool GATED>
+constexpr int smem_bytes() {
+  return DATA_BYTES + RED_BYTES + (GATED ? 0 : STG_BYTES) + 1024 + 256 + 2 * 4 * kGroupSlots;
+}
+static_assert(smem_bytes<false>() <= 227 * 1024, "shared memory of one CTA");
 constexpr unsigned long long kTeardownLimitNs = 1000000000ull;
 
 // A scale fetched ahead of its use: the asm keeps the load where it is written
@@ -199,7 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* a_smem = base;
   uint8_t* b_smem = base + STAGES * A_BYTES;
   float* red = reinterpret_cast<float*>(base + DATA_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + DATA_BYTES + RED_BYTES);
+  uint8_t* stg_all = base + DATA_BYTES + RED_BYTES;
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(base + DATA_BYTES + RED_BYTES + (GATED ? 0 : STG_BYTES));
   uint64_t* full = bars;                 // stage loaded (TMA bytes)
   uint64_t* empty = bars + STAGES;       // stage consumed by the MMAs
   uint64_t* pfull = bars + 2 * STAGES;   // partial buffer written
@@ -510,21 +522,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (hh == 0) p.sd[(size_t)row * (p.ldd / 128) + fin.f0 / 128] = s;
         }
-      } else if (ok && live && any_cols) {
-        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) + (size_t)(fin.row0 + r) * p.ldd +
-                           fin.f0 + hh * 128;
-        uint4* dst = reinterpret_cast<uint4*>(y);
+      } else if (ok && any_cols) {
+        // bf16 y: this warp's 32 rows x 128 columns go out in four rounds of 8 rows.
+        // The round's 8 lanes put their 256-byte row segments into shared memory
+        // (16-byte chunk c of row j at slot c ^ j: no bank conflicts either way),
+        // then every store instruction writes two whole segments (lanes 0-15 one row,
+        // 16-31 the next), so that the stores cover whole cache lines.
+        uint8_t* stg = stg_all + ew * (8 * 256);
+        const uint32_t stg_s = smem_u32(stg);
+        const int wrow = q * 32;                         // this warp's first row in the tile
+#pragma unroll 1
+        for (int rnd = 0; rnd < 4; ++rnd) {
+          if ((lane >> 3) == rnd) {
+            const int j = lane & 7;
 #pragma unroll
-        for (int w8 = 0; w8 < 16; ++w8) {
-          uint4 o;
-          __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+            for (int w8 = 0; w8 < 16; ++w8) {
+              uint4 o;
+              __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int c2 = w8 * 4 + j;                 // column pair
-            const float2 a = c2 < 32 ? acc_a[c2] : acc_b[c2 - 32];
-            po[j] = __floats2bfloat162_rn(a.x, a.y);
+              for (int jj = 0; jj < 4; ++jj) {
+                const int c2 = w8 * 4 + jj;              // column pair
+                const float2 a = c2 < 32 ? acc_a[c2] : acc_b[c2 - 32];
+                po[jj] = __floats2bfloat162_rn(a.x, a.y);
+              }
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               stg_s + j * 256 + ((w8 ^ j) & 15) * 16),
+                           "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+                           : "memory");
+            }
           }
-          dst[w8] = o;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = 2 * i + (lane >> 4);           // row within the round
+            const int c = lane & 15;                     // 16-byte chunk of the segment
+            uint4 o;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+                         : "r"(stg_s + j * 256 + ((c ^ j) & 15) * 16)
+                         : "memory");
+            const int tr = wrow + rnd * 8 + j;           // row within the tile
+            if (tr < fin.rows) {
+              __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.d) +
+                                 (size_t)(fin.row0 + tr) * p.ldd + fin.f0 + hh * 128;
+              reinterpret_cast<uint4*>(y)[c] = o;
+            }
+          }
+          __syncwarp();
         }
       }
       if (!GATED && p.send.n_send > 0) signal_tile_stored(p.send.done, fin.g);
@@ -585,10 +629,10 @@ cudaError_t prepare_grouped_gemm_fp8_kernels() {
   if (e == cudaSuccess) e = check_register_split<false>();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<true>());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<false>());
   return e;
 }
 
@@ -635,15 +679,17 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemmFp8Args& a, cudaStream_t st
   if (p.n_gemm < 1) return cudaErrorInvalidValue;
 
   if (a.gated) {
-    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
+    grouped_gemm_fp8_kernel<true><<<a.num_ctas, kThreads, smem_bytes<true>(), st>>>(tmA, tmW, tmWs,
+                                                                                    p);
   } else if (p.send.n_send == 0) {
-    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, SMEM_BYTES, st>>>(tmA, tmW, tmWs, p);
+    grouped_gemm_fp8_kernel<false><<<a.num_ctas, kThreads, smem_bytes<false>(), st>>>(tmA, tmW,
+                                                                                      tmWs, p);
   } else {
     // the senders wait on the tiles: every CTA must be resident at once
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.num_ctas, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem_bytes<false>();
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
