@@ -531,25 +531,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* stg = stg_all + ew * (8 * 256);
         const uint32_t stg_s = smem_u32(stg);
         const int wrow = q * 32;                         // this warp's first row in the tile
+        uint32_t pk[64];                                 // the row's 128 bf16, packed in pairs
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          const float2 a = c2 < 32 ? acc_a[c2] : acc_b[c2 - 32];
+          const __nv_bfloat162 b = __floats2bfloat162_rn(a.x, a.y);
+          pk[c2] = *reinterpret_cast<const uint32_t*>(&b);
+        }
 #pragma unroll 1
         for (int rnd = 0; rnd < 4; ++rnd) {
           if ((lane >> 3) == rnd) {
             const int j = lane & 7;
 #pragma unroll
-            for (int w8 = 0; w8 < 16; ++w8) {
-              uint4 o;
-              __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                const int c2 = w8 * 4 + jj;              // column pair
-                const float2 a = c2 < 32 ? acc_a[c2] : acc_b[c2 - 32];
-                po[jj] = __floats2bfloat162_rn(a.x, a.y);
-              }
+            for (int w8 = 0; w8 < 16; ++w8)
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                                stg_s + j * 256 + ((w8 ^ j) & 15) * 16),
-                           "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+                           "r"(pk[4 * w8]), "r"(pk[4 * w8 + 1]), "r"(pk[4 * w8 + 2]),
+                           "r"(pk[4 * w8 + 3])
                            : "memory");
-            }
           }
           __syncwarp();
 #pragma unroll

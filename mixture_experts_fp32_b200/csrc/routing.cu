@@ -471,11 +471,12 @@ __global__ void __launch_bounds__(256) reduce_pairs_kernel(const float* __restri
 }
 
 // FP8 path, activation quantisation: a warp takes up to four 1x128 groups of one
-// valid token (their loads issued together), computes for each s = amax / 448 (1 if
-// amax = 0) and the e4m3 codes of x / s (fp32 division, round to nearest even,
-// saturating), once per token, and stores codes and scale straight into every
-// permuted row the token occupies (its k routed rows and the shared one, from the
-// inverse permutation): the GEMM's activation rows are written once, with no
+// valid token (eight lanes a group, 16 consecutive values a lane, loads issued
+// together), computes for each s = amax / 448 (1 if amax = 0) and the e4m3 codes of
+// x / s (fp32 division, round to nearest even, saturating), once per token, and
+// stores codes and scale straight into every permuted row the token occupies (its k
+// routed rows and the shared one, from the inverse permutation), one 512-byte store
+// of the warp per row: the GEMM's activation rows are written once, with no
 // per-token copy to gather from.
 constexpr int kQuantGroupsPerWarp = 4;
 
@@ -495,38 +496,55 @@ __global__ void __launch_bounds__(256) quant_scatter_kernel(const __nv_bfloat16*
     const int g0 = (int)(wc - (long long)t * chunks) * kQuantGroupsPerWarp;
     if (valid != nullptr && !valid[t]) continue;
     const int ng = min(kQuantGroupsPerWarp, groups - g0);
-    uint2 raw[kQuantGroupsPerWarp];
-#pragma unroll
-    for (int u = 0; u < kQuantGroupsPerWarp; ++u)
-      if (u < ng)
-        raw[u] = *reinterpret_cast<const uint2*>(x + (size_t)t * H + (size_t)(g0 + u) * 128 +
-                                                 lane * 4);
+    // lane l takes 16 consecutive values of group u = l / 8 (eight lanes a group), so
+    // that a row's four groups leave the warp as one 512-byte store per row
+    const int u = lane >> 3;
+    const bool act = u < ng;
+    const size_t col = (size_t)g0 * 128 + (size_t)lane * 16;
+    uint4 raw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    if (act) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + col);
+      raw[0] = src[0];
+      raw[1] = src[1];
+    }
     int rows[kMaxTopK + 1];
 #pragma unroll
     for (int j = 0; j < kMaxTopK + 1; ++j) rows[j] = j < ks ? inv[(size_t)t * ks + j] : -1;
+    float v[16];
 #pragma unroll
-    for (int u = 0; u < kQuantGroupsPerWarp; ++u) {
-      if (u >= ng) break;
-      const int g = g0 + u;
-      const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw[u].x);
-      const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw[u].y);
-      const float v[4] = {__low2float(p0), __high2float(p0), __low2float(p1), __high2float(p1)};
-      float a = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t w4[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-      const float s = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
-      uint32_t packed = 0;
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w4[i]);
+        v[8 * h + 2 * i] = __low2float(pr);
+        v[8 * h + 2 * i + 1] = __high2float(pr);
+      }
+    }
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    if (!act) continue;
+    const float sc = a > 0.f ? __fdiv_rn(a, 448.f) : 1.f;
+    uint32_t packed[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      packed[w] = 0;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[i], s), __NV_SATFINITE, __NV_E4M3)
-                  << (8 * i);
+        packed[w] |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[4 * w + i], sc), __NV_SATFINITE,
+                                                     __NV_E4M3)
+                     << (8 * i);
+    }
+    const uint4 q = make_uint4(packed[0], packed[1], packed[2], packed[3]);
 #pragma unroll
-      for (int j = 0; j < kMaxTopK + 1; ++j) {
-        const int r = rows[j];
-        if (r < 0) continue;
-        *reinterpret_cast<uint32_t*>(xp + (size_t)r * H + (size_t)g * 128 + lane * 4) = packed;
-        if (lane == 0) sxp[(size_t)r * groups + g] = s;
-      }
+    for (int j = 0; j < kMaxTopK + 1; ++j) {
+      const int r = rows[j];
+      if (r < 0) continue;
+      *reinterpret_cast<uint4*>(xp + (size_t)r * H + col) = q;
+      if ((lane & 7) == 0) sxp[(size_t)r * groups + g0 + u] = sc;
     }
   }
 }
