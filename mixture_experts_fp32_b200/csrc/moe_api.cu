@@ -145,7 +145,7 @@ MOE_EXPORT moe_status moe_plan_create(const moe_config* cfg, moe_plan_t* plan,
   p->off_done = take(sizeof(unsigned int) * (E + 2));
   p->off_wsplit = take(2 * 3 * (size_t)moe::router_padded_experts((int)E) * H);
   p->off_rscratch = take(sizeof(int) * (size_t)moe::route_scratch_ints((int)T, (int)E));
-  p->off_partial = take(sizeof(float) * moe::kRouterSplitMax * T * E);
+  p->off_partial = take(sizeof(float) * (size_t)moe::router_partial_rows((int)T) * E);
   p->off_logits = take(sizeof(float) * T * E);
   p->off_ids = take(sizeof(int) * T * c.top_k_max);
   p->off_w = take(sizeof(float) * T * c.top_k_max);
@@ -260,7 +260,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
   record(dbg, 0, st);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned int), st) != cudaSuccess) return MOE_ERR_CUDA;
   int splits = 1, kb_per_split = H / 64;
-  moe::router_split_plan(T, E, H, plan->num_sms, &splits, &kb_per_split);
+  moe::router_split_plan(T, E, H, plan->num_sms, moe::router_partial_rows(c.max_tokens),
+                         &splits, &kb_per_split);
   // the router weights' bf16 split: the caller's (written once by
   // moe_split_router_weights), else made here in the workspace
   const __nv_bfloat16* w3 = static_cast<const __nv_bfloat16*>(wts->router_split);
@@ -275,7 +276,8 @@ static moe_status forward_impl(moe_plan_t plan, const moe_weights* wts, const vo
   if (s != MOE_OK) return s;
   record(dbg, 1, st);
   s = check_launch(moe::launch_topk(partial, splits, wts->router_b, valid, T, E, k, c.renormalize,
-                                    logits, ids, w, st));
+                                    dbg != nullptr && dbg->logits != nullptr ? logits : nullptr,
+                                    ids, w, st));
   if (s != MOE_OK) return s;
   record(dbg, 2, st);
   s = check_launch(moe::launch_route(ids, valid, T, E, k, S, eb, ee, goff, perm, inv, rowtok,

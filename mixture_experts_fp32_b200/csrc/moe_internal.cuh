@@ -15,6 +15,13 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 constexpr int kRouterSplitMax = 16;
+// The router's partial sums [splits, T, E] get room for kRouterSplitMax splits of
+// max(max_tokens, kRouterSplitRows) rows, so that small batches may split K further
+// (more CTAs streaming the router weights).
+constexpr int kRouterSplitRows = 512;
+inline int router_partial_rows(int max_tokens) {
+  return kRouterSplitMax * (max_tokens > kRouterSplitRows ? max_tokens : kRouterSplitRows);
+}
 constexpr int kMaxTpRanks = 8;
 
 // Where the combine writes token t's result: the layer's bf16 output row, or
@@ -149,7 +156,8 @@ cudaError_t launch_reduce_pairs(const float* slab, int k, int n_extra, int rows,
                                 cudaStream_t st);
 cudaError_t prepare_grouped_gemm_kernels();
 const moe_config* plan_config(const moe_plan_s* plan);
-void router_split_plan(int T, int E, int H, int num_sms, int* splits, int* kb_per_split);
+void router_split_plan(int T, int E, int H, int num_sms, int partial_rows, int* splits,
+                       int* kb_per_split);
 
 // ---------------------------------------------------------------- device side
 

@@ -219,12 +219,15 @@ bool map_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
 
 int router_padded_experts(int E) { return (E + 15) / 16 * 16; }
 
-void router_split_plan(int T, int E, int H, int num_sms, int* splits_out, int* kb_per_split_out) {
+void router_split_plan(int T, int E, int H, int num_sms, int partial_rows, int* splits_out,
+                       int* kb_per_split_out) {
   const int kb_total = H / RBK;
   const int tiles = ((T + RBM - 1) / RBM) * ((router_padded_experts(E) + RBN - 1) / RBN);
   int splits = (2 * num_sms + tiles - 1) / tiles;
   if (splits < 1) splits = 1;
-  if (splits > kRouterSplitMax) splits = kRouterSplitMax;
+  // as many splits as the partial-sum buffer holds rows of this batch
+  const int cap = T > 0 ? partial_rows / T : kRouterSplitMax;
+  if (splits > cap) splits = cap;
   if (splits > kb_total) splits = kb_total;
   const int per = (kb_total + splits - 1) / splits;
   *kb_per_split_out = per;

@@ -39,19 +39,40 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
     return;
   }
 
+  // the splits are added in order, each element's sum starting from 0; a split's loads
+  // for all of the lane's experts go out together (one round trip per split, not one
+  // per split and expert)
   float v[8];
   uint32_t avail = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     v[i] = 0.f;
+    if (i < per_lane && lane + 32 * i < E) avail |= 1u << i;
+  }
+  for (int sp0 = 0; sp0 < splits; sp0 += 4) {
+    float pv[4][8];                       // four splits' loads before any of their adds
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float* prow = partial + ((size_t)(sp0 + b) * T + t) * E + lane;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        pv[b][i] = (sp0 + b < splits && ((avail >> i) & 1u)) ? prow[32 * i] : 0.f;
+    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      if (sp0 + b < splits) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += pv[b][i];
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
     const int e = lane + 32 * i;
-    if (i < per_lane && e < E) {
-      float s = 0.f;
-      for (int sp = 0; sp < splits; ++sp) s += partial[((size_t)sp * T + t) * E + e];
-      if (bias != nullptr) s += bias[e];
-      v[i] = s;
-      if (logits_out != nullptr) logits_out[(size_t)t * E + e] = s;
-      avail |= 1u << i;
+    if ((avail >> i) & 1u) {
+      if (bias != nullptr) v[i] += bias[e];
+      if (logits_out != nullptr) logits_out[(size_t)t * E + e] = v[i];
+    } else {
+      v[i] = 0.f;
     }
   }
 
