@@ -9,8 +9,9 @@
 //   in chunks of 1024; inside a chunk, a shared-memory bitmap per expert (one
 //   bit per token) gives each pair its rank by population counts.
 // gather_rows_kernel: x_perm[r] = x[row_token[r]] with 16-byte vectors.
-// combine_kernel: out[t] = bf16( sum_j w[t,j] y[inv[t,j]] + y[inv[t,k]] ),
-//   y in fp32, summed in fp32 in ascending j, shared expert last; padding rows get +0.0
+// combine_flat_kernel (fp32 y) / combine_kernel (bf16 y, a block per token):
+//   out[t] = bf16( sum_j w[t,j] y[inv[t,j]] + y[inv[t,k]] ),
+//   summed in fp32 in ascending j, shared expert last; padding rows get +0.0
 //   (the combine phase, [SGLang] MoE 모델을 위한 Single Batch Overlap 기법,
 //   §들어가며; the fused shared expert, Step3 推論最適化 (MI308X vs H20),
 //   §最適化技術).  For tensor parallelism the same sum (this rank's share of the
@@ -396,6 +397,74 @@ __global__ void __launch_bounds__(256, sizeof(YT) == 2 ? 3 : 1)
   }
 }
 
+template <typename YT, bool F32OUT, int MAXKS>
+__global__ void __launch_bounds__(256)
+    combine_flat_kernel(const YT* __restrict__ y, int H, const int* __restrict__ inv,
+                   const float* __restrict__ w, const uint8_t* __restrict__ valid, int T, int k,
+                   int S, const CombineOut co) {
+  // one (token, 8-column vector) pair per thread and step: every thread of the grid
+  // busy whatever the mix of valid and padding rows; a warp's 32 vectors mostly
+  // share their token, so its index loads are broadcasts.  (With bf16 expert
+  // outputs and nine rows a token, the per-token form below is faster.)
+  const int ks = k + S;
+  const int nv = H / 8;
+  const long long total = (long long)T * nv;
+  for (long long task = (long long)blockIdx.x * blockDim.x + threadIdx.x; task < total;
+       task += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(task / nv);
+    const int v = (int)(task - (long long)t * nv);
+    const bool ok = valid == nullptr || valid[t];
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (ok) {
+      const int* rows = inv + (size_t)t * ks;
+      const float* wts = w + (size_t)t * k;
+      // every row's vector is requested before the sums (one round trip, not k+S),
+      // and the sums keep their order: j ascending, then the shared expert
+      // (named registers rather than an array, which the compiler put in local memory)
+      static_assert(kMaxTopK == 8, "one register set per possible row below");
+      const YT* yv = y + (size_t)v * 8;
+#define MOE_LD(J)                                              \
+  Vec8<YT> r##J;                                               \
+  const int row##J = (J < MAXKS && J < ks) ? rows[J] : -1;     \
+  if (row##J >= 0) r##J = ld8(yv + (size_t)row##J * H);
+      MOE_LD(0) MOE_LD(1) MOE_LD(2) MOE_LD(3) MOE_LD(4) MOE_LD(5) MOE_LD(6) MOE_LD(7) MOE_LD(8)
+#undef MOE_LD
+#define MOE_FMA(J)                                                                 \
+  if (J < MAXKS && J < k && row##J >= 0) {                                         \
+    const float wj = wts[J];                                                       \
+    _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] =                         \
+        fmaf(wj, elem8(r##J, i), acc[i]);                                          \
+  }
+      MOE_FMA(0) MOE_FMA(1) MOE_FMA(2) MOE_FMA(3) MOE_FMA(4) MOE_FMA(5) MOE_FMA(6) MOE_FMA(7)
+#undef MOE_FMA
+      // the shared expert's row (slot k), added last
+#define MOE_SH(J)                                                                  \
+  if (J < MAXKS && S && J == k && row##J >= 0) {                                   \
+    _Pragma("unroll") for (int i = 0; i < 8; ++i) acc[i] += elem8(r##J, i);        \
+  }
+      MOE_SH(1) MOE_SH(2) MOE_SH(3) MOE_SH(4) MOE_SH(5) MOE_SH(6) MOE_SH(7) MOE_SH(8)
+#undef MOE_SH
+    }
+    if (F32OUT) {
+      const int owner = t / co.rows_per_rank, lt = t - owner * co.rows_per_rank;
+      float* base = co.dst[0];
+#pragma unroll
+      for (int r = 1; r < kMaxTpRanks; ++r)
+        if (owner == r) base = co.dst[r];
+      float4* dst32 =
+          reinterpret_cast<float4*>(base + ((size_t)co.slot * co.rows_per_rank + lt) * H);
+      dst32[2 * v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst32[2 * v + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+      uint4 o;
+      __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      reinterpret_cast<uint4*>(co.bf16 + (size_t)t * H)[v] = o;
+    }
+  }
+}
+
 // Owner side of the tensor-parallel reduction: the slab holds one fp32 partial
 // row per rank for each of this rank's rows; they are summed in rank order (the
 // same order on every owner) and rounded once to bf16.
@@ -606,15 +675,29 @@ void launch_combine_rows(const YT* y, int H, const int* inv, const float* w,
                                                                   S, out);
 }
 
+template <bool F32OUT>
+void launch_combine_flat(const float* y, int H, const int* inv, const float* w,
+                         const uint8_t* valid, int T, int k, int S, const CombineOut& out,
+                         cudaStream_t st) {
+  const long long blocks = ((long long)T * (H / 8) + 255) / 256;
+  const int grid = (int)(blocks < 1 ? 1 : blocks > 148 * 16 ? 148 * 16 : blocks);
+  if (k + S <= 4)
+    combine_flat_kernel<float, F32OUT, 4><<<grid, 256, 0, st>>>(y, H, inv, w, valid, T, k, S,
+                                                                out);
+  else
+    combine_flat_kernel<float, F32OUT, kMaxTopK + 1><<<grid, 256, 0, st>>>(y, H, inv, w, valid,
+                                                                          T, k, S, out);
+}
+
+// fp32 expert outputs (bf16 weights): one (token, vector) pair a thread, which keeps a
+// batch that is mostly padding rows (the DP-padded gather) as busy as a full one
 cudaError_t launch_combine(const float* y, int H, const int* inv, const float* w,
                            const uint8_t* valid, int T, int k, int S, const CombineOut& out,
                            cudaStream_t st) {
-  int grid = T < 148 * 16 ? T : 148 * 16;
-  if (grid < 1) grid = 1;
   if (out.bf16 != nullptr)
-    launch_combine_rows<float, false>(y, H, inv, w, valid, T, k, S, out, grid, st);
+    launch_combine_flat<false>(y, H, inv, w, valid, T, k, S, out, st);
   else
-    launch_combine_rows<float, true>(y, H, inv, w, valid, T, k, S, out, grid, st);
+    launch_combine_flat<true>(y, H, inv, w, valid, T, k, S, out, st);
   return cudaGetLastError();
 }
 
