@@ -29,6 +29,7 @@ namespace moe {
 namespace {
 
 constexpr int kChunk = 1024;
+constexpr int kScatterSplit = 4;   // blocks that share one chunk's scatter
 
 // Pairs routed to experts outside [eb, ee) (the experts this call computes; all of
 // them, 0..E, unless a rank of an expert-parallel layer owns only a range) are left
@@ -161,8 +162,9 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
 // The same permutation for many chunks in parallel: (1) each chunk counts its
 // pairs per expert and its valid tokens, (2) one block turns the counts into
 // group offsets and per-chunk bases (expert-major, chunk-minor, so tokens stay
-// ascending inside an expert), (3) each chunk ranks and scatters its pairs.
-// Identical results to route_kernel.
+// ascending inside an expert), (3) each chunk ranks and scatters its pairs, four
+// blocks to a chunk (each builds the chunk's bitmaps and stores the pairs of a
+// quarter of its tokens).  Identical results to route_kernel.
 __global__ void __launch_bounds__(1024, 1) route_count_kernel(const int* __restrict__ ids,
                                                               const uint8_t* __restrict__ valid,
                                                               int T, int E, int k, int eb, int ee,
@@ -242,7 +244,8 @@ __global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
     int* __restrict__ row_token, unsigned int* status) {
   __shared__ uint32_t bits[kMaxExperts][32];
   __shared__ int wvalid[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, c = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = blockIdx.x / kScatterSplit, part = blockIdx.x % kScatterSplit;
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
   __syncthreads();
@@ -252,7 +255,9 @@ __global__ void __launch_bounds__(1024, 1) route_scatter_kernel(
   const uint32_t vb = __ballot_sync(0xffffffffu, ok);
   if (lane == 0) wvalid[warp] = __popc(vb);
   __syncthreads();
-  if (t >= T) return;
+  // every block of the chunk builds its bitmaps; each stores the pairs of its own
+  // share of the chunk's tokens (the scattered stores are spread over more SMs)
+  if (tid / (kChunk / kScatterSplit) != part || t >= T) return;
   const int ks = k + S;
   if (!ok) {
     for (int j = 0; j < ks; ++j) inv[(size_t)t * ks + j] = -1;
@@ -647,9 +652,9 @@ cudaError_t launch_route(const int* ids, const uint8_t* valid, int T, int E, int
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // set_bits reports a bad expert id once in the count pass; the scatter pass skips it quietly
-  route_scatter_kernel<<<nchunks, 1024, 0, st>>>(ids, valid, T, E, k, S, eb, ee, chunk_base,
-                                                 vbase, group_offsets, perm, inv, row_token,
-                                                 status);
+  route_scatter_kernel<<<nchunks * kScatterSplit, 1024, 0, st>>>(
+      ids, valid, T, E, k, S, eb, ee, chunk_base, vbase, group_offsets, perm, inv, row_token,
+      status);
   return cudaGetLastError();
 }
 
