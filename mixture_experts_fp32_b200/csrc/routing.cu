@@ -41,7 +41,7 @@ __device__ __forceinline__ void set_bits(uint32_t (*bits)[32], const int* ids, c
     for (int j = 0; j < k; ++j) {
       const int e = ids[(size_t)t * k + j];
       if (e < 0 || e >= E) {
-        atomicOr(status, MOE_DEV_BAD_EXPERT_ID);
+        if (status != nullptr) atomicOr(status, MOE_DEV_BAD_EXPERT_ID);
         continue;
       }
       if (e >= eb && e < ee) atomicOr(&bits[e][warp], 1u << lane);
@@ -108,16 +108,19 @@ __global__ void __launch_bounds__(1024, 1) route_kernel(const int* __restrict__ 
   const int routed_rows = group_offsets[E];
   const int ks = k + S;
 
-  // pass 2: ranks, permutation, inverse, row -> token
+  // pass 2: ranks, permutation, inverse, row -> token (with one chunk, the bitmaps of
+  // pass 1 are still in place)
   for (int c = 0; c < nchunks; ++c) {
-    for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
-    __syncthreads();
     const int t = c * kChunk + tid;
-    set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, status);
     const bool ok = t < T && (valid == nullptr || valid[t]);
     const uint32_t vb = __ballot_sync(0xffffffffu, ok);
-    if (lane == 0) wvalid[warp] = __popc(vb);
-    __syncthreads();
+    if (nchunks > 1) {
+      for (int i = tid; i < E * 32; i += blockDim.x) bits[i >> 5][i & 31] = 0u;
+      __syncthreads();
+      set_bits(bits, ids, valid, T, E, k, eb, ee, t, warp, lane, nullptr);
+      if (lane == 0) wvalid[warp] = __popc(vb);
+      __syncthreads();
+    }
     if (t < T) {
       if (ok) {
         for (int j = 0; j < k; ++j) {
