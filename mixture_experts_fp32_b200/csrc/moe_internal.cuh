@@ -18,7 +18,7 @@ constexpr int kRouterSplitMax = 16;
 // The router's partial sums [splits, T, E] get room for kRouterSplitMax splits of
 // max(max_tokens, kRouterSplitRows) rows, so that small batches may split K further
 // (more CTAs streaming the router weights).
-constexpr int kRouterSplitRows = 512;
+constexpr int kRouterSplitRows = 256;
 inline int router_partial_rows(int max_tokens) {
   return kRouterSplitMax * (max_tokens > kRouterSplitRows ? max_tokens : kRouterSplitRows);
 }

@@ -17,6 +17,9 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
 }
 
+// NB: splits whose loads are issued together (4 for a few splits, where fewer
+// registers keep more warps resident; 8 when the router split K many ways)
+template <int NB>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ partial, int splits,
                                                    const float* __restrict__ bias,
                                                    const uint8_t* __restrict__ valid, int T, int E,
@@ -39,9 +42,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
     return;
   }
 
-  // the splits are added in order, each element's sum starting from 0; a split's loads
-  // for all of the lane's experts go out together (one round trip per split, not one
-  // per split and expert)
+  // the splits are added in order, each element's sum starting from 0; the loads of
+  // NB splits for all of the lane's experts go out together (one round trip per NB
+  // splits, not one per split and expert)
   float v[8];
   uint32_t avail = 0;
 #pragma unroll
@@ -49,17 +52,17 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
     v[i] = 0.f;
     if (i < per_lane && lane + 32 * i < E) avail |= 1u << i;
   }
-  for (int sp0 = 0; sp0 < splits; sp0 += 4) {
-    float pv[4][8];                       // four splits' loads before any of their adds
+  for (int sp0 = 0; sp0 < splits; sp0 += NB) {
+    float pv[NB][8];                      // NB splits' loads before any of their adds
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < NB; ++b) {
       const float* prow = partial + ((size_t)(sp0 + b) * T + t) * E + lane;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         pv[b][i] = (sp0 + b < splits && ((avail >> i) & 1u)) ? prow[32 * i] : 0.f;
     }
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < NB; ++b)
       if (sp0 + b < splits) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] += pv[b][i];
@@ -133,8 +136,13 @@ cudaError_t launch_topk(const float* partial, int splits, const float* bias, con
                         int T, int E, int k, int renorm, float* logits_out, int* ids, float* w,
                         cudaStream_t st) {
   const int warps = 8;
-  topk_kernel<<<(T + warps - 1) / warps, warps * 32, 0, st>>>(partial, splits, bias, valid, T, E,
-                                                              k, renorm, logits_out, ids, w);
+  const int grid = (T + warps - 1) / warps;
+  if (splits > 4)
+    topk_kernel<8><<<grid, warps * 32, 0, st>>>(partial, splits, bias, valid, T, E, k, renorm,
+                                                logits_out, ids, w);
+  else
+    topk_kernel<4><<<grid, warps * 32, 0, st>>>(partial, splits, bias, valid, T, E, k, renorm,
+                                                logits_out, ids, w);
   return cudaGetLastError();
 }
 
