@@ -174,9 +174,19 @@ __global__ void __launch_bounds__(RThreads, 1)
         float v[16];
         tmem_ld_16(tmem_base + ((uint32_t)(q * 32) << 16) + c0, v);
         if (t < p.T) {
+          // 16-byte stores where four experts of the row exist (the row is E floats,
+          // 16-byte aligned when E is a multiple of 4), single floats otherwise
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            if (e0 + c0 + c < p.E) out[c0 + c] = v[c];
+          for (int c = 0; c < 16; c += 4) {
+            if ((p.E & 3) == 0 && e0 + c0 + c + 3 < p.E) {
+              *reinterpret_cast<float4*>(out + c0 + c) =
+                  make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (e0 + c0 + c + i < p.E) out[c0 + c + i] = v[c + i];
+            }
+          }
         }
       }
     }
