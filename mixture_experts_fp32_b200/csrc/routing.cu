@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(256)
   // one (token, 8-column vector) pair per thread and step: every thread of the grid
   // busy whatever the mix of valid and padding rows; a warp's 32 vectors mostly
   // share their token, so its index loads are broadcasts.  (With bf16 expert
-  // outputs and nine rows a token, the per-token form below is faster.)
+  // outputs and nine rows a token, the per-token combine_kernel is faster.)
   const int ks = k + S;
   const int nv = H / 8;
   const long long total = (long long)T * nv;
