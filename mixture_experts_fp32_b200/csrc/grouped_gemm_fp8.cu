@@ -52,7 +52,9 @@
 // (setmaxnreg.dec).  Warpgroups 1 and 2 (8 warps) promote and finish, with the
 // registers warpgroup 0 released: warp w reads TMEM lanes 32*(w%4)... and one
 // half of the tile's columns, 128 fp32 accumulators a thread.  Every wait is
-// bounded and suspends rather than spins.
+// bounded; the two on the partial-buffer hand-off (the MMA issuer's for a free
+// buffer, the epilogue's for a written one) poll instead of suspending, the others
+// suspend.
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
@@ -102,7 +104,7 @@ __device__ __forceinline__ float ldg_ahead(const float* p) {
 }
 
 // Two 16-column TMEM loads without a wait, and the wait that ties the
-// registers: no use of r can be scheduled before the wait.
+// registers of two such pairs: no use of r or q can be scheduled before it.
 __device__ __forceinline__ void tmem_ld_2x16(uint32_t a0, uint32_t a1, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -117,17 +119,24 @@ __device__ __forceinline__ void tmem_ld_2x16(uint32_t a0, uint32_t a1, uint32_t 
       : "r"(a0), "r"(a1)
       : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait_tied(uint32_t (&r)[32]) {
+
+__device__ __forceinline__ void tmem_ld_wait_tied2(uint32_t (&r)[32], uint32_t (&q)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
                  "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
                  "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
                  "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
                  "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31])
+                 "+r"(r[30]), "+r"(r[31]), "+r"(q[0]), "+r"(q[1]), "+r"(q[2]), "+r"(q[3]),
+                 "+r"(q[4]), "+r"(q[5]), "+r"(q[6]), "+r"(q[7]), "+r"(q[8]), "+r"(q[9]),
+                 "+r"(q[10]), "+r"(q[11]), "+r"(q[12]), "+r"(q[13]), "+r"(q[14]), "+r"(q[15]),
+                 "+r"(q[16]), "+r"(q[17]), "+r"(q[18]), "+r"(q[19]), "+r"(q[20]), "+r"(q[21]),
+                 "+r"(q[22]), "+r"(q[23]), "+r"(q[24]), "+r"(q[25]), "+r"(q[26]), "+r"(q[27]),
+                 "+r"(q[28]), "+r"(q[29]), "+r"(q[30]), "+r"(q[31])
                :
                : "memory");
 }
+
 // acc[base .. base+15] += s * (32 loaded columns, as 16 pairs)
 __device__ __forceinline__ void promote16(float2 (&acc)[32], int base, const uint32_t (&r)[32],
                                           float2 s) {
@@ -341,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb, ++kcount) {
           const uint32_t pb = kcount & 1u;
           const uint32_t use = kcount >> 1;
-          if (!mbar_wait_sleep(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns,
-                               p.status, p.timeout_bit) ||
+          if (!mbar_wait_bounded(smem_u32(&pempty[pb]), (use & 1u) ^ 1u, p.wait_limit_ns,
+                                 p.status, p.timeout_bit) ||
               !mbar_wait_sleep(smem_u32(&full[stage]), phase, p.wait_limit_ns, p.status,
                                p.timeout_bit)) {
             ok = false;
@@ -444,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (GATED) nxt_wb = ldg_ahead(cur.swb + kb + 1);
         }
         if (ok)
-          ok = mbar_wait_sleep_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns, p.status,
-                                    p.timeout_bit);
+          ok = mbar_wait_bounded_warp(smem_u32(&pfull[pb]), use & 1u, p.wait_limit_ns,
+                                      p.status, p.timeout_bit);
         if (!ok) continue;
         tc_fence_after();
         // the partial buffer goes back to the MMA issuer as soon as it has been read
@@ -460,20 +469,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t ra[32], rb[32];
           // gated: gate columns hh*64 .. +63 -> acc_a, up columns 128 + hh*64 .. -> acc_b;
           // down: columns hh*128 .. +63 -> acc_a, +64 .. +127 -> acc_b (one scale block).
+          // Two TMEM round trips of 64 columns; the buffer is released after the second
+          // (the last 32 FMAs after the release).
           const uint32_t c0 = GATED ? tl + hh * 64 : tl + hh * 128;
           const uint32_t c1 = GATED ? tl + 128 + hh * 64 : tl + hh * 128 + 64;
           tmem_ld_2x16(c0, c0 + 16, ra);
-          tmem_ld_wait_tied(ra);
           tmem_ld_2x16(c1, c1 + 16, rb);
+          tmem_ld_wait_tied2(ra, rb);
           promote16(acc_a, 0, ra, sa2);
-          tmem_ld_wait_tied(rb);
-          tmem_ld_2x16(c0 + 32, c0 + 48, ra);
           promote16(acc_b, 0, rb, sb2);
-          tmem_ld_wait_tied(ra);
+          tmem_ld_2x16(c0 + 32, c0 + 48, ra);
           tmem_ld_2x16(c1 + 32, c1 + 48, rb);
-          promote16(acc_a, 16, ra, sa2);
-          tmem_ld_wait_tied(rb);
+          tmem_ld_wait_tied2(ra, rb);
           release();
+          promote16(acc_a, 16, ra, sa2);
           promote16(acc_b, 16, rb, sb2);
         } else {
           release();
