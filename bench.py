@@ -775,6 +775,12 @@ def cpu_baseline(w, inp, gpu, target_s: float):
     return out
 
 
+def microbatch_rows(n_ranks: int, rows: int, lo: int, hi: int):
+    """Rows of the gathered batch that one micro-batch holds: rows [lo, hi) of every
+    rank's block of `rows`, in rank order (what the micro-batch's all_gather builds)."""
+    return [r * rows + i for r in range(n_ranks) for i in range(lo, hi)]
+
+
 def tp_reference_rows(d, w, rank: int, n_ranks: int, rows: int, ranges, dev):
     """This rank's rows [rank * rows, (rank + 1) * rows) as one GPU's plain forward
     computes them, before the layer is sharded: one forward per micro-batch, over the
@@ -792,8 +798,7 @@ def tp_reference_rows(d, w, rank: int, n_ranks: int, rows: int, ranges, dev):
                        d.get("ws_down"), d.get("ss_gate_up"), d.get("ss_down"))
     mine = torch.empty(rows, w.H, dtype=torch.bfloat16, device=dev)
     for lo, hi in ranges:
-        idx = torch.cat([torch.arange(r * rows + lo, r * rows + hi, device=dev)
-                         for r in range(n_ranks)])
+        idx = torch.tensor(microbatch_rows(n_ranks, rows, lo, hi), device=dev)
         out = torch.empty(len(idx), w.H, dtype=torch.bfloat16, device=dev)
         plan.forward(wts, d["x"][idx].contiguous(), d["valid"][idx].contiguous(), w.k, out)
         mine[lo:hi] = out[rank * (hi - lo):(rank + 1) * (hi - lo)]

@@ -54,6 +54,18 @@ def test_launch_count_per_step():
     assert bench.launches_per_step(synth.WORKLOADS["fp8_prefill"]) == 9
 
 
+def test_microbatch_rows_follow_the_all_gather():
+    # two ranks of 4 rows, micro-batches [0, 2) and [2, 4): each gathers its slice of
+    # every rank in rank order
+    assert bench.microbatch_rows(2, 4, 0, 2) == [0, 1, 4, 5]
+    assert bench.microbatch_rows(2, 4, 2, 4) == [2, 3, 6, 7]
+    # together they cover the gathered batch once
+    rows = sorted(bench.microbatch_rows(3, 5, 0, 2) + bench.microbatch_rows(3, 5, 2, 5))
+    assert rows == list(range(15))
+    # one micro-batch is the whole gathered batch in order
+    assert bench.microbatch_rows(4, 3, 0, 3) == list(range(12))
+
+
 def test_tp_launch_count_per_step():
     w = synth.WORKLOADS["step3_decode"]
     # one micro-batch: the layer over 8 x 32 gathered rows (7 kernels) + the owner's sum
